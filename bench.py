@@ -1,0 +1,523 @@
+#!/usr/bin/env python3
+"""Benchmark of DeltaLog decode on B200: one JSON line on rank 0.
+
+A step is one merge cycle of an R-layer stack of identical decode layers:
+C tokens, each through all R layers in turn (append + read-out per layer),
+with each layer's merge after its C-th append -- one CUDA-graph launch
+(dl_cycle_launch).  R rotating layers keep every base read cold in L2
+(working set >= 4x the 126 MB L2).  Throughput is decode tokens per second
+through one layer (B sequences x C tokens x R layers per step), the
+amortised latency is the step time / (C R).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--layers R] [--impl native|reference]
+
+Under torchrun (N > 1) every rank runs its own replica (independent
+batches, no collective on the data path); rank 0 prints the aggregate with
+the time taken as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = ("amortized µs/token state update, decode tok/s, HBM GB/s vs roofline, "
+          "bytes written/token")
+DEFAULT_WORKLOAD = "gdn-b128-h16-d128-c8"
+L2_BYTES = 126 * 1000 * 1000
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------ ranks ------
+
+def rank_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world, backend, timeout_s=120):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend,
+                                timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def reduce_over_ranks(elapsed_ms: float, units: float, device=None):
+    """(max elapsed over ranks, sum of units over ranks); identity at N = 1."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(elapsed_ms), float(units)
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------ byte model ------
+
+def bytes_model(w):
+    """Algorithmic HBM bytes per head (read, write) of each kernel.
+
+    append(L): base read once, L logged entries (key, value factor,
+    log-decay), the token's inputs; writes the output and one log entry.
+    merge(L): base read + L entries, base written.  eager: state read and
+    written, inputs read, output written."""
+    ie = 2 if w.in_dtype == "bf16" else 4
+    oe = 2 if w.out_dtype == "bf16" else 4
+    ue = ie if w.op == 2 else 4
+    m = w.m
+    S = 4 * w.dk * w.dv
+    E = w.dk * ie + w.dv * ue + 4 * m
+    I = (2 * w.dk + w.dv) * ie + 4 * m + (0 if w.op == 2 else 4) + (4 * w.dk if w.op == 2 else 0)
+    O = w.dv * oe
+
+    def append(L):
+        return S + L * E + I, O + E
+
+    def merge(L):
+        return S + L * E, S
+
+    eager = (S + I, S + O)
+    C = w.C
+    cyc_r = sum(append(L)[0] for L in range(C)) + merge(C)[0]
+    cyc_w = sum(append(L)[1] for L in range(C)) + merge(C)[1]
+    return {"S": S, "E": E, "I": I, "O": O, "append": append, "merge": merge,
+            "eager": eager, "token_read": cyc_r / C, "token_write": cyc_w / C}
+
+
+# --------------------------------------------------------- clocks -------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a thread."""
+
+    def __init__(self, torch_device, period_s=0.005):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.h = None
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            props = __import__("torch").cuda.get_device_properties(torch_device)
+            h = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    h = N.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+                except Exception:
+                    h = None
+            if h is None:
+                h = N.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.h = h
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.error = repr(e)
+
+    def _run(self):
+        N = self.N
+        fn = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            N.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM),
+                                     int(fn(self.h))))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.h is not None:
+            self.t.join()
+
+    def summary(self):
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": getattr(self, "error", "nvml unavailable")}
+        busy = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        reasons = set()
+        for _, r in busy:
+            for bit, name in _REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return dict(PEAKS_FALLBACK)
+
+
+def recorded_traffic(workload_name):
+    """Per-launch DRAM bytes of the append kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"append_kernel_{workload_name}.md")
+    src = os.path.join(ROOT, "recurrent_state_head_b200", "csrc", "kernels.cuh")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+        m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        if m_sha and m_b and m_sha.group(1) == sha:
+            return float(m_b.group(1))
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------- CPU oracle -----
+
+def cpu_oracle_sample(w, target_s=12.0, seed=99):
+    """Time the fp64 oracle's base+log decode on a bounded sample of heads
+    of the workload (one merge cycle of C tokens); returns tok/s in the
+    GPU's unit (head-tokens per second / H), the threads used and a note."""
+    import oracle
+    from recurrent_state_head_b200 import synth
+
+    threads = max(1, len(os.sched_getaffinity(0)))
+    rng = np.random.default_rng(seed)
+
+    def run(n_heads):
+        heads = np.sort(rng.choice(w.heads, size=min(n_heads, w.heads), replace=False))
+        ti = synth.tokens(w, 0, w.C, heads=heads)
+        S0 = synth.initial_state(w).reshape(w.heads, w.dk, w.dv)[heads]
+        bon = synth.bonus(w)
+        bon = None if bon is None else bon[heads % w.H]
+        g = ti.g.astype(np.float64)
+        if g.ndim == 2:
+            g = g[:, :, None]
+        st = oracle.LogState(w.op, S0, w.C)
+        t0 = time.perf_counter()
+        oracle.deltalog_run(st, ti.q64, ti.k64, ti.v64,
+                            None if w.op == 2 else ti.beta.astype(np.float64), g, bon,
+                            w.scale, n_threads=threads)
+        return time.perf_counter() - t0, len(heads)
+
+    probe_heads = max(threads, 8)
+    dt, n = run(probe_heads)
+    per_head = dt / n
+    n_heads = int(max(probe_heads, min(w.heads, target_s / max(per_head, 1e-9))))
+    dt, n = run(n_heads)
+    head_tokens = n * w.C
+    return {"value": head_tokens / dt / w.H, "unit": "tok/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} of {w.heads} heads x {w.C} tokens (one merge cycle), "
+                      f"fp64 base+log oracle, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------ native ----
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    from recurrent_state_head_b200 import binding as B
+    from recurrent_state_head_b200 import device as D
+    from recurrent_state_head_b200 import synth
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    B.lib()                                   # fail loudly if the library is missing
+
+    w = synth.WORKLOADS[args.workload]
+    R = args.layers
+    C, NH = w.C, w.heads
+    bm = bytes_model(w)
+    stream = torch.cuda.current_stream(dev)
+
+    # --- state and inputs of R independent layers (replica-specific seeds)
+    layers, xs, outs, eager_S = [], [], [], []
+    for l in range(R):
+        lid = rank * R + l
+        S0 = synth.initial_state(w, layer=lid)
+        bon = synth.bonus(w, layer=lid)
+        layers.append(D.DecodeLayer(w, S0, bon, device=dev))
+        xs.append(D.to_device(synth.tokens(w, 0, C, layer=lid, want64=False), w, dev))
+        outs.append(layers[-1].new_out(C))
+        if args.eager:
+            eager_S.append(layers[-1].base.clone())
+    working_set = R * (NH * bm["S"] + NH * C * bm["E"])
+    ios = [[(xs[l]["q"][t], xs[l]["k"][t], xs[l]["v"][t],
+             None if w.op == synth.RWKV6 else xs[l]["beta"][t], xs[l]["g"][t], outs[l][t])
+            for l in range(R)] for t in range(C)]
+    cycle = B.Cycle([L_.handle for L_ in layers], ios)
+    kernels_per_step = cycle.kernels
+
+    # --- timed region: K cycle launches
+    for _ in range(args.warmup):
+        cycle.launch(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            cycle.launch(stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    elapsed_ms = ev0.elapsed_time(ev1)
+    tokens_local = w.B * C * R * args.steps          # decode tokens through one layer
+    max_ms, tokens_all = reduce_over_ranks(elapsed_ms, tokens_local, dev)
+    ms_per_step = max_ms / args.steps
+    tok_s = tokens_all / (max_ms / 1e3)
+    us_per_token = ms_per_step * 1e3 / (C * R)
+    gbs = NH * (bm["token_read"] + bm["token_write"]) * C * R / (ms_per_step / 1e3) / 1e9
+
+    # --- per-kernel durations (same stream, same cold rotation), non-graph
+    prof_layers = []
+    for l in range(R):
+        lid = rank * R + l
+        prof_layers.append(D.DecodeLayer(w, synth.initial_state(w, layer=lid),
+                                         synth.bonus(w, layer=lid), device=dev, auto_merge=0))
+    n_prof = max(2, min(args.steps, 10))
+    app_ms = {L: [] for L in range(C)}
+    mrg_ms = []
+    for it in range(n_prof + 1):
+        evs = []
+        for t in range(C):
+            for l in range(R):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                prof_layers[l].step(xs[l], t, outs[l][t], stream)
+                b.record(stream)
+                evs.append(("a", t, a, b))
+                if t == C - 1:
+                    a2, b2 = (torch.cuda.Event(enable_timing=True),
+                              torch.cuda.Event(enable_timing=True))
+                    a2.record(stream)
+                    prof_layers[l].merge(stream)
+                    b2.record(stream)
+                    evs.append(("m", t, a2, b2))
+        torch.cuda.synchronize(dev)
+        if it == 0:
+            continue                                   # warm-up cycle
+        for kind, t, a, b in evs:
+            (app_ms[t] if kind == "a" else mrg_ms).append(a.elapsed_time(b))
+    app_avg_ms = statistics.mean([x for L in range(C) for x in app_ms[L]])
+    app_bytes_avg = NH * statistics.mean([sum(bm["append"](L)) for L in range(C)])
+    mrg_avg_ms = statistics.mean(mrg_ms)
+    peaks = measured_peaks()
+    achieved = app_bytes_avg / (app_avg_ms / 1e3) / 1e9
+    traffic = recorded_traffic(args.workload)
+
+    result = {
+        "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "op": ["gdn", "kda", "rwkv6"][w.op], "B": w.B,
+                   "H": w.H, "dk": w.dk, "dv": w.dv, "C": C, "layers_rotated": R,
+                   "inputs": f"q/k/v {w.in_dtype}, out {w.out_dtype}, fp32 state",
+                   "l2": f"inputs larger than L2: {R} rotating layers, working set "
+                         f"{working_set / 1e6:.0f} MB vs L2 {L2_BYTES / 1e6:.0f} MB",
+                   "step": f"one CUDA-graph merge cycle: {C} tokens x {R} layers appends "
+                           f"+ {R} merges",
+                   "parallelism": f"replicas{world}"},
+        "us_per_token": us_per_token,
+        "hbm_gbs": gbs,
+        "hbm_frac": gbs / peaks["hbm_gbs"],
+        "bytes_written_per_token": NH * bm["token_write"],
+        "bytes_read_per_token": NH * bm["token_read"],
+        "kernels": {"append_avg_us": app_avg_ms * 1e3, "merge_avg_us": mrg_avg_ms * 1e3,
+                    "append_us_by_L": [statistics.mean(app_ms[L]) * 1e3 for L in range(C)]},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "kernel": "append_kernel",
+                     "peak_source": peaks["source"]},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    # --- eager dense baseline, same layers and rotation, graph-captured
+    if args.eager:
+        cfg = D.config_of(w)
+        bon = [L_.bonus for L_ in layers]
+        g_eager = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g_eager, stream=side):
+                for t in range(C):
+                    for l in range(R):
+                        beta = None if w.op == synth.RWKV6 else xs[l]["beta"][t]
+                        B.dl_eager_step(cfg, eager_S[l], xs[l]["q"][t], xs[l]["k"][t],
+                                        xs[l]["v"][t], beta, xs[l]["g"][t], bon[l],
+                                        outs[l][t], side)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            g_eager.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g_eager.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1) / args.steps
+        e_read, e_write = bm["eager"]
+        result["eager"] = {
+            "us_per_token": e_ms * 1e3 / (C * R),
+            "tok_s": w.B * C * R / (e_ms / 1e3),
+            "hbm_gbs": NH * (e_read + e_write) * C * R / (e_ms / 1e3) / 1e9,
+            "bytes_written_per_token": NH * e_write,
+            "write_ratio_vs_deltalog": e_write / bm["token_write"],
+            "speedup_deltalog": (e_ms * 1e3 / (C * R)) / us_per_token,
+        }
+        result["eager"]["hbm_frac"] = result["eager"]["hbm_gbs"] / peaks["hbm_gbs"]
+        del g_eager
+
+    # --- end to end through the public API with host buffers
+    if args.e2e:
+        names = ("q", "k", "v", "beta", "g")
+        host_in = [{n: xs[l][n].cpu().pin_memory() for n in names} for l in range(R)]
+        host_out = [torch.empty(outs[l].shape, dtype=outs[l].dtype).pin_memory()
+                    for l in range(R)]
+        h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        for _ in range(max(1, args.warmup)):
+            for l in range(R):
+                for n in names:
+                    xs[l][n].copy_(host_in[l][n], non_blocking=True)
+            cycle.launch(stream)
+            for l in range(R):
+                host_out[l].copy_(outs[l], non_blocking=True)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            for l in range(R):
+                for n in names:
+                    xs[l][n].copy_(host_in[l][n], non_blocking=True)
+            cycle.launch(stream)
+            for l in range(R):
+                host_out[l].copy_(outs[l], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        e_max, e_tok = reduce_over_ranks(e0.elapsed_time(e1), tokens_local, dev)
+        result["e2e"] = {"value": e_tok / (e_max / 1e3), "unit": "tok/s",
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        result["cpu_baseline"] = cpu_oracle_sample(w)
+    cycle.close()
+    return result
+
+
+# ---------------------------------------------------------- reference ---
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: host cores, bounded samples."""
+    from recurrent_state_head_b200 import synth
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    per_step_s = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, target_s=per_step_s)
+    vals, samples = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_oracle_sample(w, target_s=per_step_s)
+        vals.append(r["value"])
+        samples.append(r)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    ms_per_step = wall * 1e3 / max(1, args.steps)
+    last = samples[-1]
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "op": ["gdn", "kda", "rwkv6"][w.op], "B": w.B,
+                   "H": w.H, "dk": w.dk, "dv": w.dv, "C": w.C,
+                   "parallelism": "host cores (oracle)"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--no-eager", dest="eager", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local_rank = rank_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_native(args, rank, world, local_rank)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    try:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * deltalog.h -- C ABI of libdeltalog.so: DeltaLog recurrent-state decode for
+ * linear-attention layers (Gated DeltaNet, KDA, RWKV6) on B200 (sm_100a).
+ *
+ * Method: "DeltaLog: Deferred Materialization of Recurrent States for Linear
+ * Attention Decoding" (arXiv 2608.15533).  Each head keeps a dense fp32 base
+ * state Sbar (d_k x d_v) plus a bounded log of at most C compact update
+ * factors; most decode steps read the base once and append one factor to the
+ * log, and a merge folds the log back into the base when it holds C entries
+ * (signal-papers page, Fig. 4 caption; gist.science technical summary,
+ * "Meccanismo Core: Base + Log" and "Implementazione del Kernel").
+ *
+ * Recurrences (per head; S is d_k x d_v, row i = key channel):
+ *   GDN   a = exp(g) scalar;  S' = a S;     u = beta (v - S'^T k);  S = S' + k u^T;  o = scale S^T q
+ *   KDA   a = exp(g) per key; S' = D(a) S;  same delta rule and readout
+ *   RWKV6 w = exp(g) per key; o = scale (S^T r + (r . (bonus * k)) v);  S = D(w) S + k v^T
+ * DeltaLog keeps, after t appends since the last merge,
+ *   S_t = D(exp(Lambda_t)) Sbar + sum_{j<=t} D(exp(Lambda_t - Lambda_j)) k_j u_j^T
+ * with Lambda_t the cumulative log-decay since the merge (inclusive of step t)
+ * and u_j the value-side factor (the delta-rule u, or the raw v for RWKV6).
+ *
+ * Conventions for every call below
+ *   - Device pointers are CUDA device (or managed) memory owned by the
+ *     caller; the library never allocates, frees or keeps device memory, and
+ *     every buffer must outlive the calls (and handles) that use it.
+ *   - Tensors are dense, row-major, with no padding.  With NH = B * H heads,
+ *     head n = b * H + h:
+ *       base / S / S_out  float  [NH, d_k, d_v]          16-byte aligned
+ *       q (r), k          in_dtype [NH, d_k]             element aligned
+ *       v                 in_dtype [NH, d_v]             element aligned
+ *       beta              float  [NH]   (GDN, KDA; NULL for RWKV6)
+ *       g (log-decay)     float  [NH] (GDN) or [NH, d_k] (KDA, RWKV6), g <= 0
+ *       bonus             float  [H, d_k]  (RWKV6 only, else NULL)
+ *       out               out_dtype [NH, d_v]
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on that stream: no host synchronisation, no
+ *     device allocation; the kernel launches can be captured in a CUDA graph.
+ *   - Arguments are checked on the host before anything is launched; on an
+ *     error nothing is launched and the handle is left as it was (except
+ *     where stated).  dl_last_error() gives a message for the calling thread.
+ *   - Supported shapes: d_k, d_v in {64, 128}; 1 <= C <= 16; B >= 0, H >= 1.
+ *     B = 0 (no heads) is accepted: nothing is launched, the log-length
+ *     schedule still advances.
+ */
+#ifndef DELTALOG_H
+#define DELTALOG_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DL_OK = 0,
+    DL_EINVAL = 1,   /* bad configuration, shape, pointer or alignment      */
+    DL_ESTATE = 2,   /* call not allowed in the current log state            */
+    DL_ECUDA = 3,    /* a CUDA runtime call or kernel launch failed          */
+    DL_ENOMEM = 4    /* host allocation failed                               */
+} dl_status;
+
+typedef enum { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2 } dl_op;
+typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
+
+typedef struct {
+    int op;          /* dl_op                                                  */
+    int B, H;        /* batch slots and heads per slot                         */
+    int dk, dv;      /* key and value width of one head's state                */
+    int C;           /* log capacity = merge interval                          */
+    int in_dtype;    /* dl_dtype of q (r), k, v and of the logged k (and v)   */
+    int out_dtype;   /* dl_dtype of out                                        */
+    float scale;     /* output scale (d_k^-1/2 for GDN/KDA is usual)           */
+    int auto_merge;  /* 1: dl_decode_step merges when the log becomes full     */
+} dl_config;
+
+typedef struct dl_handle dl_handle;   /* opaque; host memory only */
+
+/* Size in bytes of the log workspace for `cfg` (0 if cfg is invalid).
+ * Layout, each region 256-byte aligned, in this order:
+ *   K      in_dtype [NH, C, d_k]   logged keys (bit-exact copies of k)
+ *   U      [NH, C, d_v]            value factors: float (GDN, KDA), or
+ *                                  in_dtype copies of v (RWKV6)
+ *   Lambda float [NH, C, m]        cumulative log-decay since the last merge,
+ *                                  m = 1 (GDN) or d_k (KDA, RWKV6)
+ * The log is the paper's "bounded update log" (gist.science technical
+ * summary, "Meccanismo Core: Base + Log"). */
+size_t dl_log_bytes(const dl_config *cfg);
+
+/* Byte offsets of the K, U and Lambda regions inside the log workspace. */
+dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U,
+                        size_t *off_Lam);
+
+/* Create a decode handle over a caller-owned base state (device, fp32
+ * [NH, d_k, d_v], 16-byte aligned, holds S at the last merge) and log
+ * workspace (device, dl_log_bytes(cfg) bytes, 16-byte aligned).  `bonus` is
+ * the RWKV6 bonus [H, d_k] (device, float) and must be NULL otherwise.  The
+ * log starts empty (L = 0); its contents are never read before written.
+ * Errors: DL_EINVAL (config, NULL or misaligned pointer), DL_ENOMEM. */
+dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,
+                    const float *bonus, dl_handle **out);
+
+/* One decode token for all NH heads: the append + read-out step (paper:
+ * "Fase di Append", kernel stages ReplayPrep and AppendDecode, gist.science
+ * technical summary).  Reads the base once, replays the L logged factors,
+ * writes `out` (out_dtype [NH, d_v]) and appends (k, u, Lambda) at slot L;
+ * the base is not written.  Then L = L + 1, and with auto_merge the merge
+ * runs when L reaches C (L returns to 0).
+ * Errors: DL_EINVAL (NULL / misaligned pointer), DL_ESTATE (log full with
+ * auto_merge = 0; nothing launched), DL_ECUDA (launch failed; L unchanged if
+ * the append failed, L = C if only the merge launch failed). */
+dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
+                         const float *beta, const float *g, void *out, void *stream);
+
+/* Merge phase (paper: "Fase di Merge"): Sbar <- D(exp(Lambda_L)) Sbar +
+ * sum_j D(exp(Lambda_L - Lambda_j)) k_j u_j^T in place, then L = 0.
+ * A no-op when L = 0.  Errors: DL_ECUDA. */
+dl_status dl_merge(dl_handle *h, void *stream);
+
+/* Write the logical state (base + replayed log) to S_out (device fp32
+ * [NH, d_k, d_v], 16-byte aligned, must not overlap the base); base and log
+ * are left untouched.  With L = 0 this copies the base.
+ * Errors: DL_EINVAL, DL_ECUDA. */
+dl_status dl_materialize(const dl_handle *h, float *S_out, void *stream);
+
+/* Eager dense step (the in-house dense baseline; paper: eager decoding that
+ * materialises and writes back the full state every token, signal-papers
+ * page Fig. 3/4 captions): reads and rewrites S (device fp32
+ * [NH, d_k, d_v]) and writes out.  cfg->C and cfg->auto_merge are ignored.
+ * Errors: DL_EINVAL, DL_ECUDA. */
+dl_status dl_eager_step(const dl_config *cfg, float *S, const void *q, const void *k,
+                        const void *v, const float *beta, const float *g,
+                        const float *bonus, void *out, void *stream);
+
+/* Current log length L (0 <= L <= C), or -1 for a NULL handle. */
+int dl_log_len(const dl_handle *h);
+
+/* Release the handle (host memory only).  NULL is accepted. */
+void dl_destroy(dl_handle *h);
+
+/* ------------------------------------------------------- merge cycle ---- */
+/* One merge cycle of several layers as a single CUDA graph (paper: split-
+ * replay ablation "with CUDA Graph replay", latencies amortised over one
+ * merge cycle, signal-papers page Fig. 9 caption).  The graph holds, token
+ * by token, the append of every layer and, after each layer's C-th append,
+ * that layer's merge: n_layers * (C + 1) kernels.
+ *
+ * `io` is [C][n_layers] (token-major): the device pointers of each
+ * (token, layer) step, laid out as for dl_decode_step.  All layers must have
+ * the same C, auto_merge = 1, and L = 0 when the cycle is launched; they are
+ * back at L = 0 afterwards.  The graph captures the pointers: new inputs are
+ * written into the same buffers between launches. */
+typedef struct {
+    const void *q, *k, *v;
+    const float *beta, *g;
+    void *out;
+} dl_step_io;
+
+typedef struct dl_cycle dl_cycle;
+
+/* Errors: DL_EINVAL (mixed C, bad pointer), DL_ESTATE, DL_ECUDA, DL_ENOMEM. */
+dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_io *io,
+                          dl_cycle **out);
+/* Launch one cycle on `stream`.  DL_ESTATE if any layer has L != 0. */
+dl_status dl_cycle_launch(dl_cycle *cy, void *stream);
+/* Kernels in one launch of the cycle. */
+int dl_cycle_kernels(const dl_cycle *cy);
+void dl_cycle_destroy(dl_cycle *cy);
+
+/* ------------------------------------------------------------ errors ---- */
+const char *dl_strerror(dl_status s);
+/* Detail of the last error on the calling thread ("" if none). */
+const char *dl_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTALOG_H */

@@ -1,0 +1,107 @@
+"""Device memory for DeltaLog decode: PyTorch allocates, the library computes.
+
+``DecodeLayer`` owns one layer's base state, log workspace and (RWKV6)
+bonus as torch tensors and a ``binding.Handle`` over them;
+``to_device`` moves seeded host inputs (``synth.TokenInputs``) to the GPU
+in the library's dtypes.  Nothing here computes any part of the recurrence.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .synth import RWKV6, TokenInputs, Workload
+
+DTYPE_CODE = {"f32": B.DL_F32, "bf16": B.DL_BF16}
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def host_tensor(a: np.ndarray, dtype: str) -> torch.Tensor:
+    """Wrap a host array stored as `dtype` (bf16 arrives as raw uint16 bits)."""
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+
+
+def to_device(ti: TokenInputs, w: Workload, device="cuda", pin: bool = False):
+    """Stacked token inputs as tensors: q, k [T, NH, dk]; v [T, NH, dv];
+    beta [T, NH]; g [T, NH, m].  With device=None the tensors stay on the host
+    (pinned if `pin`)."""
+    T = ti.q.shape[0]
+    NH = w.heads
+    out = {
+        "q": host_tensor(ti.q, w.in_dtype).reshape(T, NH, w.dk),
+        "k": host_tensor(ti.k, w.in_dtype).reshape(T, NH, w.dk),
+        "v": host_tensor(ti.v, w.in_dtype).reshape(T, NH, w.dv),
+        "beta": torch.from_numpy(np.ascontiguousarray(ti.beta, dtype=np.float32)).reshape(T, NH),
+        "g": torch.from_numpy(np.ascontiguousarray(ti.g, dtype=np.float32)).reshape(T, NH, w.m),
+    }
+    if device is None:
+        if pin:
+            out = {k: v.pin_memory() for k, v in out.items()}
+        return out
+    return {k: v.to(device, non_blocking=True) for k, v in out.items()}
+
+
+def config_of(w: Workload, C=None, auto_merge=1) -> B.dl_config:
+    return B.make_config(w.op, w.B, w.H, w.dk, w.dv, w.C if C is None else C,
+                         DTYPE_CODE[w.in_dtype], DTYPE_CODE[w.out_dtype], w.scale, auto_merge)
+
+
+class DecodeLayer:
+    """One layer of DeltaLog decode state on the GPU."""
+
+    def __init__(self, w: Workload, S0: np.ndarray, bonus=None, device="cuda", C=None,
+                 auto_merge=1):
+        self.w = w
+        self.cfg = config_of(w, C, auto_merge)
+        self.base = torch.from_numpy(np.ascontiguousarray(S0, dtype=np.float32)).reshape(
+            w.heads, w.dk, w.dv).to(device)
+        self.log = torch.zeros(max(B.dl_log_bytes(self.cfg), 16), dtype=torch.uint8,
+                               device=device)
+        self.bonus = (torch.from_numpy(np.ascontiguousarray(bonus, dtype=np.float32)).to(device)
+                      if w.op == RWKV6 else None)
+        self.handle = B.Handle(self.cfg, self.base, self.log, self.bonus)
+        self.out_dtype = TORCH_DTYPE[w.out_dtype]
+        self.device = device
+
+    @property
+    def L(self) -> int:
+        return self.handle.L
+
+    def new_out(self, T=None):
+        shape = (self.w.heads, self.w.dv) if T is None else (T, self.w.heads, self.w.dv)
+        return torch.empty(shape, dtype=self.out_dtype, device=self.device)
+
+    def step(self, x: dict, t: int, out: torch.Tensor, stream=None):
+        """Decode token t of the stacked inputs `x` into `out` [NH, dv]."""
+        beta = None if self.w.op == RWKV6 else x["beta"][t]
+        self.handle.decode_step(x["q"][t], x["k"][t], x["v"][t], beta, x["g"][t], out, stream)
+
+    def materialize(self, stream=None) -> torch.Tensor:
+        S = torch.empty_like(self.base)
+        self.handle.materialize(S, stream)
+        return S
+
+    def merge(self, stream=None):
+        self.handle.merge(stream)
+
+    def log_views(self):
+        """(K, U, Lambda) views of the log workspace for inspection."""
+        oK, oU, oL = B.dl_log_layout(self.cfg)
+        NH, C, dk, dv, m = self.w.heads, self.cfg.C, self.w.dk, self.w.dv, self.w.m
+        in_t = TORCH_DTYPE[self.w.in_dtype]
+        u_t = in_t if self.w.op == RWKV6 else torch.float32
+        esz = lambda t: torch.tensor([], dtype=t).element_size()  # noqa: E731
+        K = self.log[oK:oK + NH * C * dk * esz(in_t)].view(in_t).view(NH, C, dk)
+        U = self.log[oU:oU + NH * C * dv * esz(u_t)].view(u_t).view(NH, C, dv)
+        Lam = self.log[oL:oL + NH * C * m * 4].view(torch.float32).view(NH, C, m)
+        return K, U, Lam
+
+
+def eager_step(w: Workload, S: torch.Tensor, x: dict, t: int, bonus, out, stream=None):
+    cfg = config_of(w)
+    beta = None if w.op == RWKV6 else x["beta"][t]
+    B.dl_eager_step(cfg, S, x["q"][t], x["k"][t], x["v"][t], beta, x["g"][t], bonus, out,
+                    stream)

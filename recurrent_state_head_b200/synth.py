@@ -23,8 +23,10 @@ A per-token generator lets any token be drawn on its own, in any order.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -158,15 +160,16 @@ def bonus(w: Workload, layer: int = 0) -> Optional[np.ndarray]:
 
 
 def tokens(w: Workload, t0: int, n: int, layer: int = 0,
-           heads: Optional[np.ndarray] = None) -> TokenInputs:
+           heads: Optional[np.ndarray] = None, want64: bool = True) -> TokenInputs:
     """Inputs of tokens t0 .. t0+n-1 of one layer.
 
     `heads` (flat b*H + h indices) keeps only those heads; the draws are the
-    same as in the full tensors.
+    same as in the full tensors.  With want64=False the float64 views are
+    left empty (see `exact64` to widen a selection later).
     """
     B, H, dk, dv = w.B, w.H, w.dk, w.dv
-    qs, ks, vs, bs, gs, q6, k6, v6 = ([] for _ in range(8))
-    for t in range(t0, t0 + n):
+
+    def one(t):
         rng = np.random.Generator(np.random.PCG64([w.seed, layer, 2 + t]))
         q = rng.standard_normal((B, H, dk))
         k = rng.standard_normal((B, H, dk))
@@ -187,8 +190,27 @@ def tokens(w: Workload, t0: int, n: int, layer: int = 0,
         qs_, q64 = round_to(q, w.in_dtype)
         ks_, k64 = round_to(k, w.in_dtype)
         vs_, v64 = round_to(v, w.in_dtype)
-        qs.append(qs_); ks.append(ks_); vs.append(vs_)
-        q6.append(q64); k6.append(k64); v6.append(v64)
-        bs.append(beta.astype(np.float32)); gs.append(g.astype(np.float32))
+        if not want64:
+            q64 = k64 = v64 = None
+        return qs_, ks_, vs_, beta.astype(np.float32), g.astype(np.float32), q64, k64, v64
+
+    # tokens are independent streams: draw them in parallel, keep their order
+    n_workers = max(1, min(n, len(os.sched_getaffinity(0)), 16))
+    if n_workers > 1:
+        with cf.ThreadPoolExecutor(max_workers=n_workers) as ex:
+            rows = list(ex.map(one, range(t0, t0 + n)))
+    else:
+        rows = [one(t) for t in range(t0, t0 + n)]
+    qs, ks, vs, bs, gs, q6, k6, v6 = (list(c) for c in zip(*rows)) if rows else ([],) * 8
     st = np.stack
-    return TokenInputs(st(qs), st(ks), st(vs), st(bs), st(gs), st(q6), st(k6), st(v6))
+    e = np.zeros(0)
+    return TokenInputs(st(qs), st(ks), st(vs), st(bs), st(gs),
+                       st(q6) if want64 else e, st(k6) if want64 else e,
+                       st(v6) if want64 else e)
+
+
+def exact64(stored: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact float64 values of stored inputs (float32, or bf16 bits)."""
+    if dtype == "bf16":
+        return bf16_bits_to_f32(stored).astype(np.float64)
+    return np.asarray(stored, dtype=np.float32).astype(np.float64)

@@ -1,0 +1,343 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (normwise-max relative error, max|x - ref| / max|ref|, per step):
+  outputs stored in fp32   1e-4
+  outputs stored in bf16   2e-2
+  fp32 state (materialised / eager S)   1e-4
+Log-length schedule and merge points: exact.  Logged keys: bit-exact copies.
+Inputs come from the seeded generator only; the oracle sees the very same
+rounded values, widened to float64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import rel_err
+from recurrent_state_head_b200 import binding as B
+from recurrent_state_head_b200 import device as D
+from recurrent_state_head_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_STATE = 1e-4
+OPS = (synth.GDN, synth.KDA, synth.RWKV6)
+SHAPES = ((64, 64), (128, 128), (64, 128), (128, 64))
+
+
+def tol_out(w):
+    return 2e-2 if w.out_dtype == "bf16" else 1e-4
+
+
+def small(op, dk, dv, C=4, T=12, Bsz=3, H=5, in_dt="f32", out_dt="f32", seed=7,
+          init_std=0.5):
+    scale = 1.0 if op == synth.RWKV6 else dk ** -0.5
+    return synth.Workload(f"test-{op}-{dk}x{dv}", op, Bsz, H, dk, dv, C, T, in_dt, out_dt,
+                          scale, seed, init_std)
+
+
+def oracle_inputs(w, ti, heads=None, S0=None, bonus=None):
+    """Float64 oracle views of the stored inputs, optionally for some heads."""
+    T = ti.q.shape[0]
+    NH = w.heads
+    sel = (lambda a: a.reshape((T, NH) + a.shape[3:])) if heads is None else \
+        (lambda a: a.reshape((T, NH) + a.shape[3:])[:, heads])
+    q = synth.exact64(sel(ti.q), w.in_dtype)
+    k = synth.exact64(sel(ti.k), w.in_dtype)
+    v = synth.exact64(sel(ti.v), w.in_dtype)
+    beta = sel(ti.beta).astype(np.float64)
+    g = sel(ti.g).astype(np.float64)
+    if g.ndim == 2:
+        g = g[:, :, None]
+    hsel = np.arange(NH) if heads is None else np.asarray(heads)
+    S = S0.reshape(NH, w.dk, w.dv)[hsel].astype(np.float64)
+    bon = None if bonus is None else bonus[hsel % w.H].astype(np.float64)
+    return S, q, k, v, beta, g, bon
+
+
+def to_np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def run_oracle_eager(w, S, q, k, v, beta, g, bon):
+    return oracle.eager_run(w.op, S, q, k, v, None if w.op == synth.RWKV6 else beta, g, bon,
+                            w.scale)
+
+
+# --------------------------------------------------------------- eager ----
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", SHAPES)
+@pytest.mark.parametrize("dts", [("f32", "f32"), ("bf16", "bf16")])
+def test_eager_matches_oracle(op, dims, dts):
+    w = small(op, *dims, in_dt=dts[0], out_dt=dts[1])
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    S = torch.from_numpy(S0).reshape(w.heads, w.dk, w.dv).cuda()
+    bon_d = None if bonus is None else torch.from_numpy(bonus).cuda()
+    outs = torch.empty(w.T, w.heads, w.dv, dtype=D.TORCH_DTYPE[w.out_dtype], device="cuda")
+    for t in range(w.T):
+        D.eager_step(w, S, x, t, bon_d, outs[t])
+    torch.cuda.synchronize()
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
+    o = to_np(outs)
+    for t in range(w.T):
+        assert rel_err(o[t], o_ref[t]) <= tol_out(w), t
+    assert rel_err(to_np(S), S_ref) <= TOL_STATE
+
+
+# ------------------------------------------------------------ DeltaLog ----
+
+def run_deltalog(w, x, S0, bonus, C, check_every_step=None, auto_merge=1):
+    layer = D.DecodeLayer(w, S0, bonus, C=C, auto_merge=auto_merge)
+    outs = layer.new_out(w.T)
+    Ls, mats = [], []
+    for t in range(w.T):
+        layer.step(x, t, outs[t])
+        Ls.append(layer.L)
+        if check_every_step:
+            mats.append(to_np(layer.materialize()))
+    torch.cuda.synchronize()
+    return layer, outs, Ls, mats
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", SHAPES)
+@pytest.mark.parametrize("C", [1, 2, 3, 4, 8, 16])
+def test_deltalog_matches_eager_oracle(op, dims, C):
+    """Outputs every token, the logical (materialised) state after every
+    token and the log-length schedule, over two full cycles and a ragged
+    third."""
+    w = small(op, *dims, C=C, T=2 * C + 3, seed=11 + C)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True)
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    st = oracle.LogState(w.op, Sr, C)
+    _, L_ref, _ = oracle.deltalog_run(st, q, k, v, None if op == synth.RWKV6 else beta, g, bon,
+                                      w.scale)
+    assert Ls == L_ref.tolist()
+    o = to_np(outs)
+    S = Sr
+    for t in range(w.T):
+        S, o_ref = run_oracle_eager(w, S, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1],
+                                    g[t:t + 1], bon)
+        assert rel_err(o[t], o_ref[0]) <= tol_out(w), t
+        assert rel_err(mats[t], S) <= TOL_STATE, t
+    if layer.L == 0:
+        assert rel_err(to_np(layer.base), S) <= TOL_STATE
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dts", [("bf16", "bf16"), ("bf16", "f32"), ("f32", "bf16")])
+def test_deltalog_mixed_dtypes(op, dts):
+    w = small(op, 128, 128, C=4, T=11, in_dt=dts[0], out_dt=dts[1])
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, _ = run_deltalog(w, x, S0, bonus, w.C)
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
+    o = to_np(outs)
+    for t in range(w.T):
+        assert rel_err(o[t], o_ref[t]) <= tol_out(w), t
+    assert rel_err(to_np(layer.materialize()), S_ref) <= TOL_STATE
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("in_dt", ["f32", "bf16"])
+def test_log_contents(op, in_dt):
+    """Slot j: k_j bit for bit, the step's value factor (delta-rule u, or v
+    itself for RWKV6), and the cumulative log-decay since the merge."""
+    C = 6
+    w = small(op, 64, 128, C=C, T=C - 1, in_dt=in_dt, out_dt="f32")
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, _ = run_deltalog(w, x, S0, bonus, C)
+    assert layer.L == C - 1
+    K, U, Lam = layer.log_views()
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    _, _, u_ref = oracle.eager_run(w.op, Sr, q, k, v, None if op == synth.RWKV6 else beta, g,
+                                   bon, w.scale, want_u=True)
+    Kd = K.cpu()
+    kin = x["k"].cpu()
+    for j in range(C - 1):
+        if in_dt == "bf16":
+            assert torch.equal(Kd[:, j].view(torch.int16), kin[j].view(torch.int16))
+        else:
+            assert torch.equal(Kd[:, j].view(torch.int32), kin[j].view(torch.int32))
+        assert rel_err(to_np(U[:, j]), u_ref[j]) <= TOL_STATE
+        assert rel_err(to_np(Lam[:, j]), np.sum(g[:j + 1], axis=0)) <= 1e-6
+    # the base is never written by an append
+    assert torch.equal(layer.base.cpu(), torch.from_numpy(S0).reshape(w.heads, w.dk, w.dv))
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_capacity_one_equals_gpu_eager(op):
+    w = small(op, 128, 128, C=1, T=9)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, _ = run_deltalog(w, x, S0, bonus, 1)
+    assert Ls == [0] * w.T
+    S = torch.from_numpy(S0).reshape(w.heads, w.dk, w.dv).cuda()
+    bon_d = None if bonus is None else torch.from_numpy(bonus).cuda()
+    oe = torch.empty_like(outs)
+    for t in range(w.T):
+        D.eager_step(w, S, x, t, bon_d, oe[t])
+    torch.cuda.synchronize()
+    assert rel_err(to_np(outs), to_np(oe)) <= 1e-5
+    assert rel_err(to_np(layer.base), to_np(S)) <= 1e-5
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_explicit_merge_and_materialize(op):
+    """auto_merge = 0: the log fills, a further step is refused (nothing
+    launched), dl_merge folds a partial or full log; materialise leaves base
+    and log untouched."""
+    C = 5
+    w = small(op, 128, 64, C=C, T=C + 2)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer = D.DecodeLayer(w, S0, bonus, C=C, auto_merge=0)
+    outs = layer.new_out(w.T)
+    for t in range(C):
+        layer.step(x, t, outs[t])
+    assert layer.L == C
+    sentinel = torch.full_like(outs[C], 7.0)
+    with pytest.raises(B.DeltaLogError) as e:
+        layer.step(x, C, sentinel)
+    assert e.value.status == B.DL_ESTATE
+    torch.cuda.synchronize()
+    assert torch.all(sentinel == 7.0)
+    base_before = layer.base.clone()
+    log_before = layer.log.clone()
+    mat = layer.materialize()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.base, base_before) and torch.equal(layer.log, log_before)
+    layer.merge()
+    assert layer.L == 0
+    torch.cuda.synchronize()
+    assert torch.equal(layer.base, mat)
+    # a partial log: two more tokens, then merge
+    layer.step(x, C, outs[C])
+    layer.step(x, C + 1, outs[C + 1])
+    layer.merge()
+    torch.cuda.synchronize()
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
+    assert rel_err(to_np(layer.base), S_ref) <= TOL_STATE
+    for t in range(w.T):
+        assert rel_err(to_np(outs[t]), o_ref[t]) <= tol_out(w)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_cycle_graph_equals_steps(op):
+    """One graph-captured merge cycle over two layers gives the same bytes as
+    the same steps issued one by one."""
+    C = 4
+    w = small(op, 128, 128, C=C, T=C, in_dt="bf16", out_dt="bf16")
+    layers_a, layers_b, xs = [], [], []
+    for l in range(2):
+        S0 = synth.initial_state(w, layer=l)
+        bonus = synth.bonus(w, layer=l)
+        xs.append(D.to_device(synth.tokens(w, 0, C, layer=l), w))
+        layers_a.append(D.DecodeLayer(w, S0, bonus))
+        layers_b.append(D.DecodeLayer(w, S0, bonus))
+    outs_a = [layers_a[l].new_out(C) for l in range(2)]
+    outs_b = [layers_b[l].new_out(C) for l in range(2)]
+    for t in range(C):
+        for l in range(2):
+            layers_a[l].step(xs[l], t, outs_a[l][t])
+    ios = [[(xs[l]["q"][t], xs[l]["k"][t], xs[l]["v"][t],
+             None if op == synth.RWKV6 else xs[l]["beta"][t], xs[l]["g"][t], outs_b[l][t])
+            for l in range(2)] for t in range(C)]
+    cyc = B.Cycle([lb.handle for lb in layers_b], ios)
+    assert cyc.kernels == 2 * (C + 1)
+    cyc.launch()
+    torch.cuda.synchronize()
+    for l in range(2):
+        assert layers_b[l].L == 0
+        assert torch.equal(outs_a[l], outs_b[l])
+        assert torch.equal(layers_a[l].base, layers_b[l].base)
+    cyc.close()
+
+
+def test_no_heads_on_gpu():
+    w = small(synth.GDN, 128, 128, C=2, T=3, Bsz=0)
+    layer = D.DecodeLayer(w, np.zeros((0, 1, 128, 128), np.float32))
+    for t in range(3):
+        B.dl_decode_step(layer.handle.h, None, None, None, None, None, None)
+    assert layer.L == 1
+
+
+# ------------------------------------------------ full-size workloads ----
+
+def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123):
+    T = w.T if T is None else T
+    rng = np.random.default_rng(seed)
+    heads = np.unique(np.concatenate([[0, w.heads - 1],
+                                      rng.choice(w.heads, n_sample - 2, replace=False)]))
+    for l in range(layers):
+        S0 = synth.initial_state(w, layer=l)
+        bonus = synth.bonus(w, layer=l)
+        ti = synth.tokens(w, 0, T, layer=l, want64=False)
+        x = D.to_device(ti, w)
+        layer = D.DecodeLayer(w, S0, bonus)
+        outs = layer.new_out(T)
+        for t in range(T):
+            layer.step(x, t, outs[t])
+        mat = layer.materialize()
+        torch.cuda.synchronize()
+        assert torch.isfinite(outs.float()).all()
+        Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, heads=heads, S0=S0, bonus=bonus)
+        S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
+        o = to_np(outs[:, heads])
+        worst = max(rel_err(o[t], o_ref[t]) for t in range(T))
+        assert worst <= tol_out(w), worst
+        assert rel_err(to_np(mat[heads]), S_ref) <= TOL_STATE
+        del x, layer, outs, mat
+        torch.cuda.empty_cache()
+
+
+def test_full_gdn_fp32_small():
+    """The fp32 GDN case (B=1, H=2, d=64, C=4, 32 tokens from zero): every head."""
+    w = synth.WORKLOADS["gdn-b1-h2-d64-c4-fp32"]
+    S0 = synth.initial_state(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, None, w.C, check_every_step=True)
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0)
+    S = Sr
+    for t in range(w.T):
+        S, o_ref = run_oracle_eager(w, S, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1],
+                                    g[t:t + 1], None)
+        assert rel_err(to_np(outs[t]), o_ref[0]) <= 1e-4
+        assert rel_err(mats[t], S) <= TOL_STATE
+    assert Ls == [(t + 1) % w.C for t in range(w.T)]
+
+
+@pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c4",
+                                  "kda-b128-h32-d128-c8", "rwkv6-b128-h32-d64-c4",
+                                  "rwkv6-b128-h32-d64-c8"])
+def test_full_size_256_tokens(name):
+    _full_size_check(synth.WORKLOADS[name])
+
+
+@pytest.mark.parametrize("C", [1, 2, 16])
+def test_stack_largest_batch(C):
+    """The 24-layer GDN stack at its largest batch (B=512: 8192 heads per
+    layer), two of its layers, two cycles and a ragged third."""
+    w = synth.WORKLOADS[f"gdn-stack24-b512-h16-d128-c{C}"]
+    _full_size_check(w, layers=2, T=2 * C + 3)
