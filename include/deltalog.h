@@ -26,12 +26,14 @@
  *   - Tensors are dense, row-major, with no padding.  With NH = B * H heads,
  *     head n = b * H + h:
  *       base / S / S_out  float  [NH, d_k, d_v]          16-byte aligned
- *       q (r), k          in_dtype [NH, d_k]             element aligned
- *       v                 in_dtype [NH, d_v]             element aligned
- *       beta              float  [NH]   (GDN, KDA; NULL for RWKV6)
- *       g (log-decay)     float  [NH] (GDN) or [NH, d_k] (KDA, RWKV6), g <= 0
- *       bonus             float  [H, d_k]  (RWKV6 only, else NULL)
- *       out               out_dtype [NH, d_v]
+ *       q (r), k          in_dtype [NH, d_k]             16-byte aligned
+ *       v                 in_dtype [NH, d_v]             16-byte aligned
+ *       beta              float  [NH]   (GDN, KDA; ignored for RWKV6)  4-byte aligned
+ *       g (log-decay)     float  [NH] (GDN, 4-byte aligned) or [NH, d_k]
+ *                         (KDA, RWKV6, 16-byte aligned), g <= 0
+ *       bonus             float  [H, d_k]  (RWKV6 only, 16-byte aligned;
+ *                         ignored otherwise)
+ *       out               out_dtype [NH, d_v]            element aligned
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *     call is asynchronous on that stream: no host synchronisation, no
  *     device allocation; the kernel launches can be captured in a CUDA graph.
@@ -93,7 +95,8 @@ dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U,
 /* Create a decode handle over a caller-owned base state (device, fp32
  * [NH, d_k, d_v], 16-byte aligned, holds S at the last merge) and log
  * workspace (device, dl_log_bytes(cfg) bytes, 16-byte aligned).  `bonus` is
- * the RWKV6 bonus [H, d_k] (device, float) and must be NULL otherwise.  The
+ * the RWKV6 bonus [H, d_k] (device, float, 16-byte aligned; ignored for the
+ * other operators).  The
  * log starts empty (L = 0); its contents are never read before written.
  * Errors: DL_EINVAL (config, NULL or misaligned pointer), DL_ENOMEM. */
 dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,

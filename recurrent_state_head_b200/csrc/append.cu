@@ -3,13 +3,35 @@
 
 namespace dl {
 namespace {
-template <int OP, int DK, int DV>
-cudaError_t launch(const AppendParams &p, cudaStream_t s) {
-    using LC = LaunchCfg<DK, DV>;
-    const unsigned grid = (unsigned)p.NH * (DV / LC::TV);
-    append_kernel<OP, DK, DV, LC::TV, LC::NT><<<grid, LC::NT, 0, s>>>(p);
+template <int OP, int DK, int DV, int TV>
+cudaError_t launch_tv(AppendParams p, cudaStream_t s, int sms) {
+    constexpr int NT = 4 * TV;
+    static PlanCache cache;
+    auto kern = append_kernel<OP, DK, DV, TV, NT>;
+    const int ie = p.in_bf16 ? 2 : 4;
+    Plan plan;
+    cudaError_t e = cache.get(kern, NT, stage_layout<OP, DK, TV>(p.L, ie, true).bytes, &plan);
+    if (e != cudaSuccess) return e;
+    p.ns = plan.ns;
+    const long long units = (long long)p.NH * (DV / TV);
+    const int grid = (int)std::min<long long>(units, (long long)sms * plan.per_sm);
+    kern<<<grid, NT, plan.smem, s>>>(p);
     return cudaGetLastError();
 }
+
+template <int OP, int DK, int DV>
+cudaError_t launch(const AppendParams &p, cudaStream_t s) {
+    DeviceFacts f;
+    cudaError_t e = device_facts(&f);
+    if (e != cudaSuccess) return e;
+    switch (pick_tile(p.NH, DV, f.sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128>(p, s, f.sms); break;
+        case 64: return launch_tv<OP, DK, DV, 64>(p, s, f.sms);
+        default: break;
+    }
+    return launch_tv<OP, DK, DV, 32>(p, s, f.sms);
+}
+
 #define ROW(OP) {{launch<OP, 64, 64>, launch<OP, 64, 128>}, {launch<OP, 128, 64>, launch<OP, 128, 128>}}
 const append_fn table[3][2][2] = {ROW(OP_GDN), ROW(OP_KDA), ROW(OP_RWKV6)};
 #undef ROW
@@ -19,5 +41,26 @@ append_fn get_append(int op, int dk, int dv) {
     const int a = DL_DIM_INDEX(dk), b = DL_DIM_INDEX(dv);
     if (op < 0 || op > 2 || a < 0 || b < 0) return nullptr;
     return table[op][a][b];
+}
+
+cudaError_t device_facts(DeviceFacts *f) {
+    static std::mutex mu;
+    static DeviceFacts cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev].sms == 0) {
+        DeviceFacts d;
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess)
+            return e;
+        cache[dev] = d;
+    }
+    *f = cache[dev];
+    return cudaSuccess;
 }
 }  // namespace dl

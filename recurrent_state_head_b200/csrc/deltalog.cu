@@ -77,15 +77,19 @@ Layout log_layout(const dl_config *c) {
     return l;
 }
 
-// Pointers of one decode step.
+// Pointers of one decode step.  The kernels copy q, k, v (and the per-key
+// log-decay rows) with 16-byte asynchronous copies.
 dl_status check_step_ptrs(const dl_config *c, const void *q, const void *k, const void *v,
                           const float *beta, const float *g, const void *out) {
-    const size_t ie = esize(c->in_dtype), oe = esize(c->out_dtype);
+    const size_t oe = esize(c->out_dtype);
     if (!q || !k || !v || !g || !out) return fail(DL_EINVAL, "q/k/v/g/out must not be NULL");
     if (c->op != DL_RWKV6 && !beta) return fail(DL_EINVAL, "beta must not be NULL for GDN/KDA");
-    if (!aligned(q, ie) || !aligned(k, ie) || !aligned(v, ie) || !aligned(out, oe) ||
-        !aligned(g, 4) || (beta && !aligned(beta, 4)))
-        return fail(DL_EINVAL, "q/k/v/out must be element aligned, beta/g 4-byte aligned");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16))
+        return fail(DL_EINVAL, "q/k/v must be 16-byte aligned");
+    if (!aligned(g, c->op == DL_GDN ? 4 : 16))
+        return fail(DL_EINVAL, "g must be 4-byte (GDN) or 16-byte (KDA/RWKV6) aligned");
+    if (!aligned(out, oe) || (beta && !aligned(beta, 4)))
+        return fail(DL_EINVAL, "out must be element aligned, beta 4-byte aligned");
     return DL_OK;
 }
 
@@ -187,8 +191,8 @@ dl_status dl_create(const dl_config *cfg, float *base, void *log_ws, const float
         if (!base || !log_ws) return fail(DL_EINVAL, "base and log workspace must not be NULL");
         if (!aligned(base, 16) || !aligned(log_ws, 16))
             return fail(DL_EINVAL, "base and log workspace must be 16-byte aligned");
-        if (cfg->op == DL_RWKV6 && (!bonus || !aligned(bonus, 4)))
-            return fail(DL_EINVAL, "RWKV6 needs a 4-byte aligned bonus [H, d_k]");
+        if (cfg->op == DL_RWKV6 && (!bonus || !aligned(bonus, 16)))
+            return fail(DL_EINVAL, "RWKV6 needs a 16-byte aligned bonus [H, d_k]");
     }
     dl_handle *h = new (std::nothrow) dl_handle;
     if (!h) return fail(DL_ENOMEM, "host allocation of the handle failed");
@@ -256,8 +260,8 @@ dl_status dl_eager_step(const dl_config *cfg, float *S, const void *q, const voi
     if (!S || !aligned(S, 16)) return fail(DL_EINVAL, "S must be non-NULL and 16-byte aligned");
     s = check_step_ptrs(cfg, q, k, v, beta, g, out);
     if (s != DL_OK) return s;
-    if (cfg->op == DL_RWKV6 && (!bonus || !aligned(bonus, 4)))
-        return fail(DL_EINVAL, "RWKV6 needs a 4-byte aligned bonus [H, d_k]");
+    if (cfg->op == DL_RWKV6 && (!bonus || !aligned(bonus, 16)))
+        return fail(DL_EINVAL, "RWKV6 needs a 16-byte aligned bonus [H, d_k]");
     dl::EagerParams p;
     p.S = S;
     p.q = q;

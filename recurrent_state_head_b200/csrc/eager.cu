@@ -5,9 +5,10 @@ namespace dl {
 namespace {
 template <int OP, int DK, int DV>
 cudaError_t launch(const EagerParams &p, cudaStream_t s) {
-    using LC = LaunchCfg<DK, DV>;
-    const unsigned grid = (unsigned)p.NH * (DV / LC::TV);
-    eager_kernel<OP, DK, DV, LC::TV, LC::NT><<<grid, LC::NT, 0, s>>>(p);
+    // one CTA per (head, 32-column tile), tile held in registers
+    constexpr int TV = 32, NT = 128;
+    const unsigned grid = (unsigned)p.NH * (DV / TV);
+    eager_kernel<OP, DK, DV, TV, NT><<<grid, NT, 0, s>>>(p);
     return cudaGetLastError();
 }
 #define ROW(OP) {{launch<OP, 64, 64>, launch<OP, 64, 128>}, {launch<OP, 128, 64>, launch<OP, 128, 128>}}

@@ -7,14 +7,16 @@
 // with shared key-side metadata and the ReplayPrep / AppendDecode stages
 // ("Implementazione del Kernel"), operators GDN / KDA / RWKV6.
 //
-// Decomposition (all kernels): one CTA per (head, value tile).  The CTA owns
-// every key row i of its TV value columns, so the key-side contractions
-// S^T x reduce inside the CTA: each thread streams RPT rows of one 16-byte
-// column group with 128-bit loads (a warp covers 32/TPR consecutive rows of
-// TV contiguous floats), folds its rows into per-column partial sums, then a
-// shuffle pass and a shared-memory pass finish the reduction.  Nothing here
-// is a dense contraction worth a tensor core: per state element the append
-// does 2 FMAs and the merge at most C = 16, against 4 to 8 bytes of HBM.
+// Decomposition.  A work unit is one head, or one value tile of a head when
+// there are too few heads to fill the GPU (the paper's value-tile split): TV
+// value columns of all d_k rows, so the key-side contractions S^T x reduce
+// inside the CTA.  NT = 4 TV threads: TV/4 threads per row, each owning a
+// 16-byte column group, 16 row groups.  The append and merge kernels are
+// persistent and stream each unit through a ring of shared-memory stages
+// filled by cp.async; the eager kernel is one CTA per 32-column tile with
+// the tile in registers.  Nothing here is a dense contraction worth a tensor
+// core: per state element the append does 2 FMAs and the merge at most
+// C = 16, against 4 to 8 bytes of HBM traffic.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,6 +43,7 @@ struct AppendParams {
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
+    int ns;                   // pipeline stages (1..4)
 };
 
 struct MergeParams {
@@ -51,6 +54,7 @@ struct MergeParams {
     const float *logLam;
     int NH, C, L;
     int in_bf16;
+    int ns;                   // pipeline stages (1..4)
 };
 
 struct EagerParams {
@@ -102,6 +106,44 @@ __device__ __forceinline__ void copy_in(void *dst, size_t di, const void *src, s
         reinterpret_cast<uint16_t *>(dst)[di] = reinterpret_cast<const uint16_t *>(src)[si];
     else
         reinterpret_cast<float *>(dst)[di] = reinterpret_cast<const float *>(src)[si];
+}
+
+// element i of a raw vector in shared (or global) memory, either dtype
+__device__ __forceinline__ float ld_raw(const void *p, int i, int bf16) {
+    if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void copy_raw(void *dst, size_t di, const void *src, int si, int bf16) {
+    if (bf16)
+        reinterpret_cast<uint16_t *>(dst)[di] = reinterpret_cast<const uint16_t *>(src)[si];
+    else
+        reinterpret_cast<float *>(dst)[di] = reinterpret_cast<const float *>(src)[si];
+}
+
+// Asynchronous global -> shared copies (sm_80+ cp.async; completion is
+// awaited with cp.async.wait_all, a hardware wait).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Copy `bytes` (a multiple of 16; both addresses 16-byte aligned) with all
+// NT threads of the CTA.
+template <int NT>
+__device__ __forceinline__ void cp_async_bytes(void *smem, const void *gmem, int bytes) {
+    char *d = static_cast<char *>(smem);
+    const char *g = static_cast<const char *>(gmem);
+    for (int o = threadIdx.x * 16; o < bytes; o += NT * 16) cp_async16(d + o, g + o);
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -159,157 +201,299 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
+// ============================================== persistent stage pipeline ==
+//
+// The append and merge kernels are persistent: a grid of (SM count x
+// resident CTAs per SM) CTAs walks the units with a stride of gridDim.x.
+// Each unit's operands -- its base tile and every small operand -- form one
+// stage in dynamic shared memory, filled with cp.async.  `ns` stages rotate:
+// while unit n is computed from its stage, the copies of units n+1 .. n+ns-1
+// are in flight, so the HBM stream does not wait for a CTA's prologue,
+// reductions or epilogue.  All waits are cp.async.wait_group (hardware) and
+// __syncthreads.
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most n of this thread's committed copy groups are pending.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    }
+}
+
+__host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
+
+// Byte offsets of one stage (all 16-byte aligned).
+struct StageLayout {
+    int base, kin, qin, vin, g, beta, bonus, K, lam, U, bytes;
+};
+
+// Append stage for log length L: base tile [DK][TV] fp32, the token's k, q
+// rows and v tile, g, beta or bonus, and the L logged entries (keys,
+// decay snapshots, the tile's value factors).  The merge stage holds the
+// base tile and the L logged entries only.
+template <int OP, int DK, int TV>
+__host__ __device__ inline StageLayout stage_layout(int L, int ie, bool append) {
+    const int M = (OP == OP_GDN) ? 1 : DK;
+    const int ue = (OP == OP_RWKV6) ? ie : 4;
+    StageLayout s{};
+    int o = 0;
+    s.base = o; o += DK * TV * 4;
+    s.kin = o; o += append ? up16(DK * ie) : 0;
+    s.qin = o; o += append ? up16(DK * ie) : 0;
+    s.vin = o; o += append ? up16(TV * ie) : 0;
+    s.g = o; o += append ? up16(M * 4) : 0;
+    s.beta = o; o += append ? 16 : 0;
+    s.bonus = o; o += (append && OP == OP_RWKV6) ? DK * 4 : 0;
+    s.K = o; o += up16(L * DK * ie);
+    s.lam = o; o += up16(L * M * 4);
+    s.U = o; o += up16(L * TV * ue);
+    s.bytes = o;
+    return s;
+}
+
+// Copy a [rows][TV] fp32 tile (row stride DV floats) into shared memory.
+template <int DV, int TV, int NT>
+__device__ __forceinline__ void cp_tile(unsigned char *dst, const float *src, int rows) {
+    constexpr int CPR = TV / 4;                     // 16-byte chunks per row
+    if constexpr (TV == DV) {                       // whole rows: one contiguous block
+        cp_async_bytes<NT>(dst, src, rows * TV * 4);
+    } else {
+        for (int idx = threadIdx.x; idx < rows * CPR; idx += NT) {
+            const int r = idx / CPR, c = idx - r * CPR;
+            cp_async16(dst + (r * TV + c * 4) * 4, src + (size_t)r * DV + c * 4);
+        }
+    }
+}
+
+// Copy the L logged value-factor rows of one tile (row stride DV elements of
+// `ue` bytes, TV elements each) into shared memory.
+template <int DV, int TV, int NT>
+__device__ __forceinline__ void cp_logrows(unsigned char *dst, const char *src, int L, int ue) {
+    if constexpr (TV == DV) {
+        cp_async_bytes<NT>(dst, src, L * TV * ue);
+    } else {
+        const int cpr = TV * ue / 16;
+        for (int idx = threadIdx.x; idx < L * cpr; idx += NT) {
+            const int j = idx / cpr, c = idx - j * cpr;
+            cp_async16(dst + j * TV * ue + c * 16, src + (size_t)j * DV * ue + c * 16);
+        }
+    }
+}
+
+// Four consecutive elements of a raw vector in shared memory as fp32.
+__device__ __forceinline__ float4 ld_raw4(const unsigned char *p, int i, int bf16) {
+    if (bf16) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p + 2 * i);
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+    }
+    return *reinterpret_cast<const float4 *>(p + 4 * i);
+}
+
 // ====================================================== append + read-out ==
 //
-// ReplayPrep (prologue, every CTA of the head): the token's key-side read-out
-// weights Gamma_t * k and Gamma_t * q (RWKV6: Gamma_{t-1} * r), the replay
-// coefficients of the L logged entries and the self term.
-// AppendDecode: x = Sbar^T w over the CTA's value tile (one base read), log
-// replay on the value side, delta correction, output, append of u.
+// ReplayPrep (once per unit, from its stage): the decay point Lambda_t
+// (RWKV6: Lambda_{t-1}), read-out weights Gamma * k and Gamma * q (RWKV6:
+// Gamma * r), replay coefficients c_j = sum_i k_i K_j[i] e^{Lam[i] - Lam_j[i]}
+// (d_j with q) and the self term.  AppendDecode: x = Sbar^T w over the tile
+// (the one base read), value-side replay, delta correction, output, append
+// of u (and, by the first tile of each head, of k and Lambda_t).
 template <int OP, int DK, int DV, int TV, int NT>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
+    static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
-    __shared__ float s_k[DK];            // k
-    __shared__ float s_q[DK];            // q (RWKV6: r)
-    __shared__ float s_lam[DK];          // Lambda used by the replay (t, or t-1 for RWKV6)
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ float s_lr[DK];           // decay point of read-out and replay
+    __shared__ float s_k[DK];
+    __shared__ float s_q[DK];
     __shared__ float s_w[NA][DK];        // read-out weights
+    __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
-    __shared__ __align__(16) float s_red[NA * T::NW * TV];
     __shared__ float s_x[NA * TV];
+    static_assert(NA * T::NW * TV <= DK * TV, "row partials fit in the consumed base tile");
 
-    const int unit = blockIdx.x;
-    const int head = unit / T::NVT;
-    const int vt = unit - head * T::NVT;
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C;
+    const int L = p.L, C = p.C, ns = p.ns;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const int ue = (OP == OP_RWKV6) ? ie : 4;
+    const StageLayout lay = stage_layout<OP, DK, TV>(L, ie, true);
+    const int n_units = p.NH * T::NVT;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
-    const int col0 = vt * TV + col4 * 4;
 
-    // 1. start the base stream: RPT rows x 16 bytes per thread, in flight
-    //    while the prologue runs
-    const float *bh = p.base + (size_t)head * DK * DV;
-    float4 s[T::RPT];
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r) s[r] = ld_stream(bh + (size_t)(rg + r * T::RG) * DV + col0);
-
-    // 2. ReplayPrep: per-key quantities of this token
-    const size_t kq_off = (size_t)head * DK;
-    const float *lamh = p.logLam + (size_t)head * C * M;
-    for (int i = tid; i < DK; i += NT) {
-        const int x = (OP == OP_GDN) ? 0 : i;
-        const float lprev = L > 0 ? lamh[(size_t)(L - 1) * M + x] : 0.f;
-        const float lt = lprev + p.g[(size_t)head * M + x];
-        const float kf = ld_in(p.k, kq_off + i, p.in_bf16);
-        const float qf = ld_in(p.q, kq_off + i, p.in_bf16);
-        s_k[i] = kf;
-        s_q[i] = qf;
-        if (OP == OP_RWKV6) {
-            s_lam[i] = lprev;
-            s_w[0][i] = expf(lprev) * qf;
+    auto issue = [&](int unit, unsigned char *st) {
+        const int head = unit / T::NVT, vt = unit - head * T::NVT;
+        cp_tile<DV, TV, NT>(st + lay.base, p.base + (size_t)head * DK * DV + vt * TV, DK);
+        cp_async_bytes<NT>(st + lay.kin, static_cast<const char *>(p.k) + (size_t)head * DK * ie, DK * ie);
+        cp_async_bytes<NT>(st + lay.qin, static_cast<const char *>(p.q) + (size_t)head * DK * ie, DK * ie);
+        cp_async_bytes<NT>(st + lay.vin,
+                           static_cast<const char *>(p.v) + ((size_t)head * DV + vt * TV) * ie, TV * ie);
+        cp_async_bytes<NT>(st + lay.K, static_cast<const char *>(p.logK) + (size_t)head * C * DK * ie,
+                           L * DK * ie);
+        const float *lamh = p.logLam + (size_t)head * C * M;
+        if (OP == OP_GDN) {
+            if (tid == 0) cp_async4(st + lay.g, p.g + head);
+            for (int j = tid; j < L; j += NT) cp_async4(st + lay.lam + 4 * j, lamh + j);
         } else {
-            s_lam[i] = lt;
-            const float gam = expf(lt);
-            s_w[0][i] = gam * kf;
-            s_w[NA - 1][i] = gam * qf;
+            cp_async_bytes<NT>(st + lay.g, p.g + (size_t)head * DK, DK * 4);
+            cp_async_bytes<NT>(st + lay.lam, lamh, L * DK * 4);
         }
-        if (vt == 0) {
-            // append the key factor and the decay snapshot at slot L
-            copy_in(p.logK, ((size_t)head * C + L) * DK + i, p.k, kq_off + i, p.in_bf16);
-            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
-        }
-    }
-    __syncthreads();
+        if (OP == OP_RWKV6)
+            cp_async_bytes<NT>(st + lay.bonus, p.bonus + (size_t)(head % p.H) * DK, DK * 4);
+        else if (tid == NT - 1)
+            cp_async4(st + lay.beta, p.beta + head);
+        cp_logrows<DV, TV, NT>(st + lay.U,
+                               static_cast<const char *>(p.logU) + ((size_t)head * C * DV + vt * TV) * ue,
+                               L, ue);
+    };
 
-    // replay coefficients: task tau < L is log entry tau, tau == L the self term
-    {
-        const int lane = tid & 31, warp = tid >> 5;
-        const float *Kf = reinterpret_cast<const float *>(p.logK);
-        const __nv_bfloat16 *Kb = reinterpret_cast<const __nv_bfloat16 *>(p.logK);
-        for (int tau = warp; tau <= L; tau += T::NW) {
-            float a0 = 0.f, a1 = 0.f;
-            if (tau < L) {
-                const size_t kb = ((size_t)head * C + tau) * DK;
-                const float *lj = lamh + (size_t)tau * M;
-                const float gdec = (OP == OP_GDN) ? expf(s_lam[0] - lj[0]) : 1.f;
-                for (int i = lane; i < DK; i += 32) {
-                    const float kj = p.in_bf16 ? __bfloat162float(Kb[kb + i]) : Kf[kb + i];
-                    const float e = (OP == OP_GDN) ? kj : expf(s_lam[i] - lj[i]) * kj;
-                    if (OP == OP_RWKV6) {
-                        a0 += s_q[i] * e;
-                    } else {
-                        a0 += s_k[i] * e;
-                        a1 += s_q[i] * e;
-                    }
-                }
-                a0 = warp_sum(a0) * gdec;
-                a1 = warp_sum(a1) * gdec;
-                if (lane == 0) {
-                    s_coef[0][tau] = a0;
-                    if (NA == 2) s_coef[NA - 1][tau] = a1;
-                }
+    for (int s = 0; s < ns - 1; ++s) {
+        const int u = blockIdx.x + s * gridDim.x;
+        if (u < n_units) issue(u, dsm + s * lay.bytes);
+        cp_async_commit();
+    }
+
+    for (int it = 0;; ++it) {
+        const int unit = blockIdx.x + it * gridDim.x;
+        if (unit >= n_units) break;
+        {
+            const int un = unit + (ns - 1) * gridDim.x;
+            if (un < n_units) issue(un, dsm + ((it + ns - 1) % ns) * lay.bytes);
+            cp_async_commit();
+        }
+        cp_async_wait_pending(ns - 1);
+        __syncthreads();
+
+        const unsigned char *st = dsm + (it % ns) * lay.bytes;
+        const int head = unit / T::NVT, vt = unit - head * T::NVT;
+        const float *sg = reinterpret_cast<const float *>(st + lay.g);
+        const float *slam = reinterpret_cast<const float *>(st + lay.lam);
+
+        // key side: decay point, read-out weights, append of k and Lambda_t
+        if (tid < DK) {
+            const int i = tid;
+            const int x = (OP == OP_GDN) ? 0 : i;
+            const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+            const float lt = lprev + sg[x];
+            const float lr = (OP == OP_RWKV6) ? lprev : lt;
+            const float kf = ld_raw(st + lay.kin, i, p.in_bf16);
+            const float qf = ld_raw(st + lay.qin, i, p.in_bf16);
+            const float gam = expf(lr);
+            s_lr[i] = lr;
+            s_k[i] = kf;
+            s_q[i] = qf;
+            if (OP == OP_RWKV6) {
+                s_w[0][i] = gam * qf;
+                s_bk[i] = reinterpret_cast<const float *>(st + lay.bonus)[i] * kf;
             } else {
-                for (int i = lane; i < DK; i += 32) {
-                    if (OP == OP_RWKV6)
-                        a0 += s_q[i] * p.bonus[(size_t)(head % p.H) * DK + i] * s_k[i];
-                    else
-                        a0 += s_k[i] * s_q[i];
+                s_w[0][i] = gam * kf;
+                s_w[NA - 1][i] = gam * qf;
+            }
+            if (vt == 0) {
+                copy_raw(p.logK, ((size_t)head * C + L) * DK + i, st + lay.kin, i, p.in_bf16);
+                if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
+            }
+        }
+        __syncthreads();
+
+        // replay coefficients: task tau < L is log entry tau, tau == L the self term
+        {
+            const int lane = tid & 31, warp = tid >> 5;
+            for (int tau = warp; tau <= L; tau += T::NW) {
+                float a0 = 0.f, a1 = 0.f;
+                if (tau < L) {
+                    const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
+#pragma unroll
+                    for (int i = lane; i < DK; i += 32) {
+                        const float kj = ld_raw(st + lay.K, tau * DK + i, p.in_bf16);
+                        const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
+                        if (OP == OP_RWKV6) {
+                            a0 = fmaf(s_q[i], e, a0);
+                        } else {
+                            a0 = fmaf(s_k[i], e, a0);
+                            a1 = fmaf(s_q[i], e, a1);
+                        }
+                    }
+                    a0 = warp_sum(a0) * gdec;
+                    if (NA == 2) a1 = warp_sum(a1) * gdec;
+                    if (lane == 0) {
+                        s_coef[0][tau] = a0;
+                        if (NA == 2) s_coef[NA - 1][tau] = a1;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = lane; i < DK; i += 32)
+                        a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
+                    a0 = warp_sum(a0);
+                    if (lane == 0) s_self = a0;
                 }
-                a0 = warp_sum(a0);
-                if (lane == 0) s_self = a0;
             }
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // 3. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
-    float4 acc[NA];
+        // base read-out from the staged tile: x_a[c] = sum_i w_a[i] * Sbar[i][c];
+        // the row partials are then reduced through the consumed tile
+        {
+            float *tile = reinterpret_cast<float *>(dsm + (it % ns) * lay.bytes + lay.base);
+            float4 acc[NA];
 #pragma unroll
-    for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < T::RPT; ++r) {
-        const int row = rg + r * T::RG;
+            for (int r = 0; r < T::RPT; ++r) {
+                const int row = rg + r * T::RG;
+                const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + col4 * 4);
 #pragma unroll
-        for (int a = 0; a < NA; ++a) {
-            const float w = s_w[a][row];
-            acc[a].x = fmaf(w, s[r].x, acc[a].x);
-            acc[a].y = fmaf(w, s[r].y, acc[a].y);
-            acc[a].z = fmaf(w, s[r].z, acc[a].z);
-            acc[a].w = fmaf(w, s[r].w, acc[a].w);
-        }
-    }
-    reduce_rows<NA, TV, NT>(acc, s_red, s_x);
-
-    // 4. value side: log replay, delta correction, output, append of u
-    for (int c = tid; c < TV; c += NT) {
-        const int col = vt * TV + c;
-        const size_t ub = (size_t)head * C * DV + col;
-        const float vv = ld_in(p.v, (size_t)head * DV + col, p.in_bf16);
-        if (OP == OP_RWKV6) {
-            float rr = 0.f;
-            for (int j = 0; j < L; ++j)
-                rr = fmaf(s_coef[0][j], ld_in(p.logU, ub + (size_t)j * DV, p.in_bf16), rr);
-            const float o = p.scale * (s_x[c] + rr + s_self * vv);
-            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-            copy_in(p.logU, ub + (size_t)L * DV, p.v, (size_t)head * DV + col, p.in_bf16);
-        } else {
-            const float *U = reinterpret_cast<const float *>(p.logU);
-            float rk = 0.f, rq = 0.f;
-            for (int j = 0; j < L; ++j) {
-                const float uj = U[ub + (size_t)j * DV];
-                rk = fmaf(s_coef[0][j], uj, rk);
-                rq = fmaf(s_coef[1][j], uj, rq);
+                for (int a = 0; a < NA; ++a) {
+                    const float w = s_w[a][row];
+                    acc[a].x = fmaf(w, sv.x, acc[a].x);
+                    acc[a].y = fmaf(w, sv.y, acc[a].y);
+                    acc[a].z = fmaf(w, sv.z, acc[a].z);
+                    acc[a].w = fmaf(w, sv.w, acc[a].w);
+                }
             }
-            const float u = p.beta[head] * (vv - s_x[c] - rk);
-            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
-            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-            reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
+            __syncthreads();
+            reduce_rows<NA, TV, NT>(acc, tile, s_x);
         }
+
+        // value side: log replay, delta correction, output, append of u
+        if (tid < TV) {
+            const int c = tid;
+            const int col = vt * TV + c;
+            const size_t ub = (size_t)head * C * DV + col;
+            const float vv = ld_raw(st + lay.vin, c, p.in_bf16);
+            if (OP == OP_RWKV6) {
+                float rr = 0.f;
+                for (int j = 0; j < L; ++j)
+                    rr = fmaf(s_coef[0][j], ld_raw(st + lay.U, j * TV + c, p.in_bf16), rr);
+                const float o = p.scale * (s_x[c] + rr + s_self * vv);
+                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+                copy_raw(p.logU, ub + (size_t)L * DV, st + lay.vin, c, p.in_bf16);
+            } else {
+                const float *U = reinterpret_cast<const float *>(st + lay.U);
+                float rk = 0.f, rq = 0.f;
+                for (int j = 0; j < L; ++j) {
+                    const float uj = U[j * TV + c];
+                    rk = fmaf(s_coef[0][j], uj, rk);
+                    rq = fmaf(s_coef[1][j], uj, rq);
+                }
+                const float beta = *reinterpret_cast<const float *>(st + lay.beta);
+                const float u = beta * (vv - s_x[c] - rk);
+                const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+                reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
+            }
+        }
+        __syncthreads();   // the stage is refilled by a later iteration's copies
     }
+    cp_async_wait_pending(0);
 }
 
 // ================================================= merge / materialise ==
@@ -317,79 +501,103 @@ append_kernel(const AppendParams p) {
 // dst[i][c] = exp(Lambda_L[i]) base[i][c] + sum_{j<L} exp(Lambda_L[i] - Lambda_j[i]) k_j[i] u_j[c]
 // (Lambda_L = the last entry's snapshot; L = 0 copies the base).  In place
 // (dst == base) it is the merge; into another buffer it is materialise.
+// Persistent, with the same stage pipeline as the append kernel.
 template <int OP, int DK, int DV, int TV, int NT>
 __global__ void __launch_bounds__(NT)
 merge_kernel(const MergeParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    constexpr int CP = MAXC + 4;             // row pitch of the coefficient table
 
+    extern __shared__ __align__(16) unsigned char dsm[];
     __shared__ float s_gam[DK];
-    __shared__ float s_coef[DK][MAXC + 1];   // [row][entry], padded against bank conflicts
+    __shared__ __align__(16) float s_coef[DK * CP];   // [row][entry]
 
-    const int unit = blockIdx.x;
-    const int head = unit / T::NVT;
-    const int vt = unit - head * T::NVT;
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C;
+    const int L = p.L, C = p.C, ns = p.ns;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const int ue = (OP == OP_RWKV6) ? ie : 4;
+    const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+    const StageLayout lay = stage_layout<OP, DK, TV>(L, ie, false);
+    const int n_units = p.NH * T::NVT;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
-    const int col0 = vt * TV + col4 * 4;
 
-    const float *lamh = p.logLam + (size_t)head * C * M;
-    // per-row decay of the base and replay coefficients
-    for (int idx = tid; idx < DK * (L + 1); idx += NT) {
-        const int i = idx % DK, j = idx / DK;          // j == L -> base decay
-        const int x = (OP == OP_GDN) ? 0 : i;
-        const float lL = L > 0 ? lamh[(size_t)(L - 1) * M + x] : 0.f;
-        if (j == L) {
-            s_gam[i] = expf(lL);
+    auto issue = [&](int unit, unsigned char *st) {
+        const int head = unit / T::NVT, vt = unit - head * T::NVT;
+        cp_tile<DV, TV, NT>(st + lay.base, p.base + (size_t)head * DK * DV + vt * TV, DK);
+        cp_async_bytes<NT>(st + lay.K, static_cast<const char *>(p.logK) + (size_t)head * C * DK * ie,
+                           L * DK * ie);
+        const float *lamh = p.logLam + (size_t)head * C * M;
+        if (OP == OP_GDN) {
+            for (int j = tid; j < L; j += NT) cp_async4(st + lay.lam + 4 * j, lamh + j);
         } else {
-            const float kj = ld_in(p.logK, ((size_t)head * C + j) * DK + i, p.in_bf16);
-            s_coef[i][j] = expf(lL - lamh[(size_t)j * M + x]) * kj;
+            cp_async_bytes<NT>(st + lay.lam, lamh, L * DK * 4);
         }
-    }
-    // value factors of this thread's four columns, every logged entry
-    float4 uu[MAXC];
-    const size_t ub = (size_t)head * C * DV + col0;
-#pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-        if (j < L) {
-            if (OP == OP_RWKV6 && p.in_bf16) {
-                const __nv_bfloat16 *Ub = reinterpret_cast<const __nv_bfloat16 *>(p.logU);
-                const size_t o = ub + (size_t)j * DV;
-                uu[j] = make_float4(__bfloat162float(Ub[o]), __bfloat162float(Ub[o + 1]),
-                                    __bfloat162float(Ub[o + 2]), __bfloat162float(Ub[o + 3]));
-            } else {
-                uu[j] = *reinterpret_cast<const float4 *>(
-                    reinterpret_cast<const float *>(p.logU) + ub + (size_t)j * DV);
-            }
-        } else {
-            uu[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
-    __syncthreads();
+        cp_logrows<DV, TV, NT>(st + lay.U,
+                               static_cast<const char *>(p.logU) + ((size_t)head * C * DV + vt * TV) * ue,
+                               L, ue);
+    };
 
-    const float *bh = p.base + (size_t)head * DK * DV;
-    float *dh = p.dst + (size_t)head * DK * DV;
-    float4 s[T::RPT];
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV + col0);
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r) {
-        const int row = rg + r * T::RG;
-        const float gm = s_gam[row];
-        float4 o = make_float4(gm * s[r].x, gm * s[r].y, gm * s[r].z, gm * s[r].w);
-#pragma unroll
-        for (int j = 0; j < MAXC; ++j) {
-            if (j < L) {
-                const float cf = s_coef[row][j];
-                o.x = fmaf(cf, uu[j].x, o.x);
-                o.y = fmaf(cf, uu[j].y, o.y);
-                o.z = fmaf(cf, uu[j].z, o.z);
-                o.w = fmaf(cf, uu[j].w, o.w);
-            }
-        }
-        st_state(dh + (size_t)row * DV + col0, o);
+    for (int s = 0; s < ns - 1; ++s) {
+        const int u = blockIdx.x + s * gridDim.x;
+        if (u < n_units) issue(u, dsm + s * lay.bytes);
+        cp_async_commit();
     }
+
+    for (int it = 0;; ++it) {
+        const int unit = blockIdx.x + it * gridDim.x;
+        if (unit >= n_units) break;
+        {
+            const int un = unit + (ns - 1) * gridDim.x;
+            if (un < n_units) issue(un, dsm + ((it + ns - 1) % ns) * lay.bytes);
+            cp_async_commit();
+        }
+        cp_async_wait_pending(ns - 1);
+        __syncthreads();
+
+        const unsigned char *st = dsm + (it % ns) * lay.bytes;
+        const int head = unit / T::NVT, vt = unit - head * T::NVT;
+        const float *slam = reinterpret_cast<const float *>(st + lay.lam);
+
+        // per-row decay of the base and replay coefficients
+        for (int idx = tid; idx < DK * (L + 1); idx += NT) {
+            const int i = idx % DK, j = idx / DK;          // j == L -> base decay
+            const int x = (OP == OP_GDN) ? 0 : i;
+            const float lL = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+            if (j == L)
+                s_gam[i] = expf(lL);
+            else
+                s_coef[i * CP + j] = expf(lL - slam[j * M + x]) * ld_raw(st + lay.K, j * DK + i, p.in_bf16);
+        }
+        __syncthreads();
+
+        const float *tile = reinterpret_cast<const float *>(st + lay.base);
+        float *dh = p.dst + (size_t)head * DK * DV + vt * TV + col4 * 4;
+#pragma unroll 2
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            const float gm = s_gam[row];
+            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + col4 * 4);
+            float4 o = make_float4(gm * sv.x, gm * sv.y, gm * sv.z, gm * sv.w);
+            for (int j0 = 0; j0 < L; j0 += 4) {
+                const float4 cf4 = *reinterpret_cast<const float4 *>(&s_coef[row * CP + j0]);
+                const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    if (j0 + jj < L) {
+                        const float4 u = ld_raw4(st + lay.U, (j0 + jj) * TV + col4 * 4, ubf);
+                        o.x = fmaf(cf[jj], u.x, o.x);
+                        o.y = fmaf(cf[jj], u.y, o.y);
+                        o.z = fmaf(cf[jj], u.z, o.z);
+                        o.w = fmaf(cf[jj], u.w, o.w);
+                    }
+                }
+            }
+            st_state(dh + (size_t)row * DV, o);
+        }
+        __syncthreads();   // the stage is refilled by a later iteration's copies
+    }
+    cp_async_wait_pending(0);
 }
 
 // ================================================================ eager ==

@@ -3,13 +3,35 @@
 
 namespace dl {
 namespace {
-template <int OP, int DK, int DV>
-cudaError_t launch(const MergeParams &p, cudaStream_t s) {
-    using LC = LaunchCfg<DK, DV>;
-    const unsigned grid = (unsigned)p.NH * (DV / LC::TV);
-    merge_kernel<OP, DK, DV, LC::TV, LC::NT><<<grid, LC::NT, 0, s>>>(p);
+template <int OP, int DK, int DV, int TV>
+cudaError_t launch_tv(MergeParams p, cudaStream_t s, int sms) {
+    constexpr int NT = 4 * TV;
+    static PlanCache cache;
+    auto kern = merge_kernel<OP, DK, DV, TV, NT>;
+    const int ie = p.in_bf16 ? 2 : 4;
+    Plan plan;
+    cudaError_t e = cache.get(kern, NT, stage_layout<OP, DK, TV>(p.L, ie, false).bytes, &plan);
+    if (e != cudaSuccess) return e;
+    p.ns = plan.ns;
+    const long long units = (long long)p.NH * (DV / TV);
+    const int grid = (int)std::min<long long>(units, (long long)sms * plan.per_sm);
+    kern<<<grid, NT, plan.smem, s>>>(p);
     return cudaGetLastError();
 }
+
+template <int OP, int DK, int DV>
+cudaError_t launch(const MergeParams &p, cudaStream_t s) {
+    DeviceFacts f;
+    cudaError_t e = device_facts(&f);
+    if (e != cudaSuccess) return e;
+    switch (pick_tile(p.NH, DV, f.sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128>(p, s, f.sms); break;
+        case 64: return launch_tv<OP, DK, DV, 64>(p, s, f.sms);
+        default: break;
+    }
+    return launch_tv<OP, DK, DV, 32>(p, s, f.sms);
+}
+
 #define ROW(OP) {{launch<OP, 64, 64>, launch<OP, 64, 128>}, {launch<OP, 128, 64>, launch<OP, 128, 128>}}
 const merge_fn table[3][2][2] = {ROW(OP_GDN), ROW(OP_KDA), ROW(OP_RWKV6)};
 #undef ROW

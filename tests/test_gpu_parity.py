@@ -134,6 +134,32 @@ def test_deltalog_matches_eager_oracle(op, dims, C):
 
 
 @pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", SHAPES)
+@pytest.mark.parametrize("nh", [200, 300])
+def test_deltalog_tile_widths(op, dims, nh):
+    """Head counts that select each unit width of the persistent kernels (a
+    whole head per unit from two units per SM up, halved value tiles below;
+    on a 148-SM B200: 300 heads -> whole heads, 200 -> 64 columns for
+    d_v = 128).  Every head, every token, and the logical state each token."""
+    C = 4
+    w = small(op, *dims, C=C, T=2 * C + 3, Bsz=nh // 4, H=4, seed=40 + nh)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True)
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    o = to_np(outs)
+    S = Sr
+    for t in range(w.T):
+        S, o_ref = run_oracle_eager(w, S, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1],
+                                    g[t:t + 1], bon)
+        assert rel_err(o[t], o_ref[0]) <= tol_out(w), t
+        assert rel_err(mats[t], S) <= TOL_STATE, t
+    assert Ls == [(t + 1) % C for t in range(w.T)]
+
+
+@pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dts", [("bf16", "bf16"), ("bf16", "f32"), ("f32", "bf16")])
 def test_deltalog_mixed_dtypes(op, dts):
     w = small(op, 128, 128, C=4, T=11, in_dt=dts[0], out_dt=dts[1])
