@@ -2,8 +2,8 @@
 """Benchmark of DeltaLog decode on B200: one JSON line on rank 0.
 
 A step is one merge cycle of an R-layer stack of identical decode layers:
-C tokens, each through all R layers in turn (append + read-out per layer),
-with each layer's merge after its C-th append -- one CUDA-graph launch
+C tokens, each through all R layers in turn -- C-1 append + read-out steps
+and one merge-token step per layer -- as one CUDA-graph launch
 (dl_cycle_launch).  R rotating layers keep every base read cold in L2
 (working set >= 4x the 126 MB L2).  Throughput is decode tokens per second
 through one layer (B sequences x C tokens x R layers per step), the
@@ -79,13 +79,15 @@ def barrier(device=None):
 
 # ------------------------------------------------------ byte model ------
 
-def bytes_model(w):
+def bytes_model(w, fold=True):
     """Algorithmic HBM bytes per head (read, write) of each kernel.
 
     append(L): base read once, L logged entries (key, value factor,
     log-decay), the token's inputs; writes the output and one log entry.
-    merge(L): base read + L entries, base written.  eager: state read and
-    written, inputs read, output written."""
+    merge_token(L): base read and written, L entries, inputs read, output
+    written.  merge(L): base read + L entries, base written.  eager: state
+    read and written, inputs read, output written.  A merge cycle of C
+    tokens is C-1 appends + a merge-token (fold) or C appends + a merge."""
     ie = 2 if w.in_dtype == "bf16" else 4
     oe = 2 if w.out_dtype == "bf16" else 4
     ue = ie if w.op == 2 else 4
@@ -98,15 +100,21 @@ def bytes_model(w):
     def append(L):
         return S + L * E + I, O + E
 
+    def merge_token(L):
+        return S + L * E + I, S + O
+
     def merge(L):
         return S + L * E, S
 
     eager = (S + I, S + O)
     C = w.C
-    cyc_r = sum(append(L)[0] for L in range(C)) + merge(C)[0]
-    cyc_w = sum(append(L)[1] for L in range(C)) + merge(C)[1]
+    if fold:
+        cyc = [append(L) for L in range(C - 1)] + [merge_token(C - 1)]
+    else:
+        cyc = [append(L) for L in range(C)] + [merge(C)]
     return {"S": S, "E": E, "I": I, "O": O, "append": append, "merge": merge,
-            "eager": eager, "token_read": cyc_r / C, "token_write": cyc_w / C}
+            "merge_token": merge_token, "eager": eager,
+            "token_read": sum(r for r, _ in cyc) / C, "token_write": sum(x for _, x in cyc) / C}
 
 
 # --------------------------------------------------------- clocks -------
@@ -251,6 +259,90 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99):
 
 # ------------------------------------------------------------ native ----
 
+def _layers(w, R, rank, dev, mode, xs=None):
+    from recurrent_state_head_b200 import device as D
+    from recurrent_state_head_b200 import synth
+    out = []
+    for l in range(R):
+        lid = rank * R + l
+        out.append(D.DecodeLayer(w, synth.initial_state(w, layer=lid), synth.bonus(w, layer=lid),
+                                 device=dev, auto_merge=mode))
+    return out
+
+
+def _ios(w, xs, outs, R, C):
+    return [[(xs[l]["q"][t], xs[l]["k"][t], xs[l]["v"][t],
+              None if w.op == 2 else xs[l]["beta"][t], xs[l]["g"][t], outs[l][t])
+             for l in range(R)] for t in range(C)]
+
+
+def _time_graph(launch, stream, steps, warmup, dev):
+    import torch
+    for _ in range(warmup):
+        launch()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        launch()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1)
+
+
+def kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps, merge_layers=None):
+    """Per-launch device time of every kernel of a merge cycle, from CUDA
+    timing events captured between the kernels of a graph (external event
+    nodes) and replayed `reps` times on the launching stream.
+
+    layers: decode layers in one automatic merge mode (each dl_decode_step is
+    one kernel in DL_MERGE_FOLD).  merge_layers (optional): layers with
+    auto_merge off, for the separate merge kernel (dl_merge)."""
+    import torch
+    from recurrent_state_head_b200 import binding as B
+    recs = []
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    fold = layers[0].cfg.auto_merge == B.DL_MERGE_FOLD
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        e.record(side)
+        return e
+
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            prev = ev()
+            for t in range(C):
+                for l in range(R):
+                    layers[l].step(xs[l], t, outs[l][t], side)
+                    e = ev()
+                    recs.append(("merge_token" if fold and t == C - 1 else "append", t, prev, e))
+                    prev = e
+            if merge_layers is not None:
+                for t in range(C):
+                    for l in range(R):
+                        merge_layers[l].step(xs[l], t, outs[l][t], side)
+                        prev = ev()
+                for l in range(R):
+                    merge_layers[l].merge(side)
+                    e = ev()
+                    recs.append(("merge", C, prev, e))
+                    prev = e
+    stream.wait_stream(side)
+    out = {}
+    g.replay()                       # warm-up
+    torch.cuda.synchronize(dev)
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for kind, t, a, b in recs:
+            out.setdefault((kind, t), []).append(a.elapsed_time(b))
+    del g
+    return out
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     from recurrent_state_head_b200 import binding as B
@@ -267,25 +359,18 @@ def run_native(args, rank, world, local_rank):
     w = synth.WORKLOADS[args.workload]
     R = args.layers
     C, NH = w.C, w.heads
-    bm = bytes_model(w)
+    bm = bytes_model(w, fold=True)
+    bm_sep = bytes_model(w, fold=False)
     stream = torch.cuda.current_stream(dev)
+    peaks = measured_peaks()
 
     # --- state and inputs of R independent layers (replica-specific seeds)
-    layers, xs, outs, eager_S = [], [], [], []
-    for l in range(R):
-        lid = rank * R + l
-        S0 = synth.initial_state(w, layer=lid)
-        bon = synth.bonus(w, layer=lid)
-        layers.append(D.DecodeLayer(w, S0, bon, device=dev))
-        xs.append(D.to_device(synth.tokens(w, 0, C, layer=lid, want64=False), w, dev))
-        outs.append(layers[-1].new_out(C))
-        if args.eager:
-            eager_S.append(layers[-1].base.clone())
+    xs = [D.to_device(synth.tokens(w, 0, C, layer=rank * R + l, want64=False), w, dev)
+          for l in range(R)]
+    layers = _layers(w, R, rank, dev, B.DL_MERGE_FOLD)
+    outs = [L_.new_out(C) for L_ in layers]
     working_set = R * (NH * bm["S"] + NH * C * bm["E"])
-    ios = [[(xs[l]["q"][t], xs[l]["k"][t], xs[l]["v"][t],
-             None if w.op == synth.RWKV6 else xs[l]["beta"][t], xs[l]["g"][t], outs[l][t])
-            for l in range(R)] for t in range(C)]
-    cycle = B.Cycle([L_.handle for L_ in layers], ios)
+    cycle = B.Cycle([L_.handle for L_ in layers], _ios(w, xs, outs, R, C))
     kernels_per_step = cycle.kernels
 
     # --- timed region: K cycle launches
@@ -311,41 +396,22 @@ def run_native(args, rank, world, local_rank):
     us_per_token = ms_per_step * 1e3 / (C * R)
     gbs = NH * (bm["token_read"] + bm["token_write"]) * C * R / (ms_per_step / 1e3) / 1e9
 
-    # --- per-kernel durations (same stream, same cold rotation), non-graph
-    prof_layers = []
-    for l in range(R):
-        lid = rank * R + l
-        prof_layers.append(D.DecodeLayer(w, synth.initial_state(w, layer=lid),
-                                         synth.bonus(w, layer=lid), device=dev, auto_merge=0))
-    n_prof = max(2, min(args.steps, 10))
-    app_ms = {L: [] for L in range(C)}
-    mrg_ms = []
-    for it in range(n_prof + 1):
-        evs = []
-        for t in range(C):
-            for l in range(R):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                prof_layers[l].step(xs[l], t, outs[l][t], stream)
-                b.record(stream)
-                evs.append(("a", t, a, b))
-                if t == C - 1:
-                    a2, b2 = (torch.cuda.Event(enable_timing=True),
-                              torch.cuda.Event(enable_timing=True))
-                    a2.record(stream)
-                    prof_layers[l].merge(stream)
-                    b2.record(stream)
-                    evs.append(("m", t, a2, b2))
-        torch.cuda.synchronize(dev)
-        if it == 0:
-            continue                                   # warm-up cycle
-        for kind, t, a, b in evs:
-            (app_ms[t] if kind == "a" else mrg_ms).append(a.elapsed_time(b))
-    app_avg_ms = statistics.mean([x for L in range(C) for x in app_ms[L]])
-    app_bytes_avg = NH * statistics.mean([sum(bm["append"](L)) for L in range(C)])
-    mrg_avg_ms = statistics.mean(mrg_ms)
-    peaks = measured_peaks()
-    achieved = app_bytes_avg / (app_avg_ms / 1e3) / 1e9
+    # --- per-kernel durations, CUDA events inside a replayed graph
+    merge_layers = _layers(w, R, rank, dev, B.DL_MERGE_OFF)
+    kd = kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps=max(3, min(args.steps, 10)),
+                          merge_layers=merge_layers)
+    app = {t: statistics.mean(kd[("append", t)]) for t in range(C - 1) if ("append", t) in kd}
+    fold_us = statistics.mean(kd[("merge_token", C - 1)]) * 1e3 if ("merge_token", C - 1) in kd else None
+    merge_us = statistics.mean(kd[("merge", C)]) * 1e3
+    if app:
+        app_avg_ms = statistics.mean(app.values())
+        app_bytes = NH * statistics.mean([sum(bm["append"](L)) for L in app])
+        dominant = "append_kernel"
+    else:                                              # C = 1: every token is a merge-token
+        app_avg_ms = fold_us / 1e3
+        app_bytes = NH * sum(bm["merge_token"](0))
+        dominant = "append_kernel (merge-token)"
+    achieved = app_bytes / (app_avg_ms / 1e3) / 1e9
     traffic = recorded_traffic(args.workload)
 
     result = {
@@ -358,27 +424,47 @@ def run_native(args, rank, world, local_rank):
                    "inputs": f"q/k/v {w.in_dtype}, out {w.out_dtype}, fp32 state",
                    "l2": f"inputs larger than L2: {R} rotating layers, working set "
                          f"{working_set / 1e6:.0f} MB vs L2 {L2_BYTES / 1e6:.0f} MB",
-                   "step": f"one CUDA-graph merge cycle: {C} tokens x {R} layers appends "
-                           f"+ {R} merges",
+                   "step": f"one CUDA-graph merge cycle of {R} layers: {C - 1} appends + "
+                           f"1 merge-token per layer, token-major",
                    "parallelism": f"replicas{world}"},
         "us_per_token": us_per_token,
         "hbm_gbs": gbs,
         "hbm_frac": gbs / peaks["hbm_gbs"],
         "bytes_written_per_token": NH * bm["token_write"],
         "bytes_read_per_token": NH * bm["token_read"],
-        "kernels": {"append_avg_us": app_avg_ms * 1e3, "merge_avg_us": mrg_avg_ms * 1e3,
-                    "append_us_by_L": [statistics.mean(app_ms[L]) * 1e3 for L in range(C)]},
+        "kernels": {"append_us_by_L": [app[L] * 1e3 for L in sorted(app)],
+                    "append_avg_us": app_avg_ms * 1e3,
+                    "merge_token_us": fold_us, "merge_us": merge_us,
+                    "merge_gbs": NH * sum(bm["merge"](C)) / (merge_us / 1e6) / 1e9},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": traffic, "kernel": "append_kernel",
+                     "traffic": traffic, "kernel": dominant,
                      "peak_source": peaks["source"]},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if fold_us:
+        result["kernels"]["merge_token_gbs"] = \
+            NH * sum(bm["merge_token"](C - 1)) / (fold_us / 1e6) / 1e9
+    del merge_layers
+
+    # --- the same cycle with the merge as its own kernel (ablation)
+    if args.ablation:
+        sep = _layers(w, R, rank, dev, B.DL_MERGE_SEPARATE)
+        cyc_sep = B.Cycle([L_.handle for L_ in sep], _ios(w, xs, outs, R, C))
+        ms = _time_graph(lambda: cyc_sep.launch(stream), stream, args.steps, args.warmup, dev)
+        ms = ms / args.steps
+        result["separate_merge"] = {
+            "us_per_token": ms * 1e3 / (C * R),
+            "hbm_gbs": NH * (bm_sep["token_read"] + bm_sep["token_write"]) * C * R / (ms / 1e3) / 1e9,
+            "bytes_written_per_token": NH * bm_sep["token_write"]}
+        cyc_sep.close()
+        del sep
 
     # --- eager dense baseline, same layers and rotation, graph-captured
     if args.eager:
         cfg = D.config_of(w)
+        eager_S = [L_.base.clone() for L_ in layers]
         bon = [L_.bonus for L_ in layers]
         g_eager = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
@@ -392,16 +478,7 @@ def run_native(args, rank, world, local_rank):
                                         xs[l]["v"][t], beta, xs[l]["g"][t], bon[l],
                                         outs[l][t], side)
         stream.wait_stream(side)
-        for _ in range(args.warmup):
-            g_eager.replay()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            g_eager.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1) / args.steps
+        e_ms = _time_graph(g_eager.replay, stream, args.steps, args.warmup, dev) / args.steps
         e_read, e_write = bm["eager"]
         result["eager"] = {
             "us_per_token": e_ms * 1e3 / (C * R),
@@ -412,7 +489,7 @@ def run_native(args, rank, world, local_rank):
             "speedup_deltalog": (e_ms * 1e3 / (C * R)) / us_per_token,
         }
         result["eager"]["hbm_frac"] = result["eager"]["hbm_gbs"] / peaks["hbm_gbs"]
-        del g_eager
+        del g_eager, eager_S
 
     # --- end to end through the public API with host buffers
     if args.e2e:
@@ -422,28 +499,19 @@ def run_native(args, rank, world, local_rank):
                     for l in range(R)]
         h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out)
-        for _ in range(max(1, args.warmup)):
+
+        def e2e_step():
             for l in range(R):
                 for n in names:
                     xs[l][n].copy_(host_in[l][n], non_blocking=True)
             cycle.launch(stream)
             for l in range(R):
                 host_out[l].copy_(outs[l], non_blocking=True)
-        torch.cuda.synchronize(dev)
+
         barrier(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            for l in range(R):
-                for n in names:
-                    xs[l][n].copy_(host_in[l][n], non_blocking=True)
-            cycle.launch(stream)
-            for l in range(R):
-                host_out[l].copy_(outs[l], non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
+        e_ms = _time_graph(e2e_step, stream, args.steps, max(1, args.warmup), dev)
         barrier(dev)
-        e_max, e_tok = reduce_over_ranks(e0.elapsed_time(e1), tokens_local, dev)
+        e_max, e_tok = reduce_over_ranks(e_ms, tokens_local, dev)
         result["e2e"] = {"value": e_tok / (e_max / 1e3), "unit": "tok/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
@@ -499,6 +567,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--no-eager", dest="eager", action="store_false")
+    ap.add_argument("--no-ablation", dest="ablation", action="store_false",
+                    help="skip the separate-merge cycle")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args(argv)

@@ -64,6 +64,19 @@ typedef enum {
 typedef enum { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2 } dl_op;
 typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
 
+/* When the log is folded into the base (dl_config.auto_merge).  Both
+ * automatic modes give the same outputs, states and log-length schedule:
+ * L after a step is (steps since the last merge) mod C. */
+typedef enum {
+    DL_MERGE_OFF = 0,      /* never: a step with L = C fails (DL_ESTATE)      */
+    DL_MERGE_FOLD = 1,     /* the C-th token is a merge-token: one kernel
+                              reads the base once, replays the C-1 logged
+                              factors and writes the merged state, this
+                              token's update included (default)              */
+    DL_MERGE_SEPARATE = 2  /* the C-th token appends, then the merge kernel
+                              folds the full log into the base                */
+} dl_merge_mode;
+
 typedef struct {
     int op;          /* dl_op                                                  */
     int B, H;        /* batch slots and heads per slot                         */
@@ -72,7 +85,7 @@ typedef struct {
     int in_dtype;    /* dl_dtype of q (r), k, v and of the logged k (and v)   */
     int out_dtype;   /* dl_dtype of out                                        */
     float scale;     /* output scale (d_k^-1/2 for GDN/KDA is usual)           */
-    int auto_merge;  /* 1: dl_decode_step merges when the log becomes full     */
+    int auto_merge;  /* dl_merge_mode                                          */
 } dl_config;
 
 typedef struct dl_handle dl_handle;   /* opaque; host memory only */
@@ -106,11 +119,14 @@ dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,
  * "Fase di Append", kernel stages ReplayPrep and AppendDecode, gist.science
  * technical summary).  Reads the base once, replays the L logged factors,
  * writes `out` (out_dtype [NH, d_v]) and appends (k, u, Lambda) at slot L;
- * the base is not written.  Then L = L + 1, and with auto_merge the merge
- * runs when L reaches C (L returns to 0).
+ * the base is not written.  Then L = L + 1.  The token that brings L to C
+ * merges: with DL_MERGE_FOLD it is the merge-token (the merged state,
+ * this token included, is written over the base by the same kernel), with
+ * DL_MERGE_SEPARATE the merge kernel runs after its append; either way L
+ * returns to 0.
  * Errors: DL_EINVAL (NULL / misaligned pointer), DL_ESTATE (log full with
- * auto_merge = 0; nothing launched), DL_ECUDA (launch failed; L unchanged if
- * the append failed, L = C if only the merge launch failed). */
+ * DL_MERGE_OFF; nothing launched), DL_ECUDA (launch failed; L unchanged if
+ * the first kernel failed, L = C if only the separate merge failed). */
 dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
                          const float *beta, const float *g, void *out, void *stream);
 
@@ -144,13 +160,14 @@ void dl_destroy(dl_handle *h);
 /* One merge cycle of several layers as a single CUDA graph (paper: split-
  * replay ablation "with CUDA Graph replay", latencies amortised over one
  * merge cycle, signal-papers page Fig. 9 caption).  The graph holds, token
- * by token, the append of every layer and, after each layer's C-th append,
- * that layer's merge: n_layers * (C + 1) kernels.
+ * by token, every layer's step; the C-th token of a layer is its
+ * merge-token (DL_MERGE_FOLD: n_layers * C kernels) or its append followed
+ * by its merge (DL_MERGE_SEPARATE: n_layers * (C + 1) kernels).
  *
  * `io` is [C][n_layers] (token-major): the device pointers of each
  * (token, layer) step, laid out as for dl_decode_step.  All layers must have
- * the same C, auto_merge = 1, and L = 0 when the cycle is launched; they are
- * back at L = 0 afterwards.  The graph captures the pointers: new inputs are
+ * the same C, an automatic merge mode, and L = 0 when the cycle is launched;
+ * they are back at L = 0 afterwards.  The graph captures the pointers: new inputs are
  * written into the same buffers between launches. */
 typedef struct {
     const void *q, *k, *v;

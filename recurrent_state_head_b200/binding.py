@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libdeltalog.so")
 DL_OK, DL_EINVAL, DL_ESTATE, DL_ECUDA, DL_ENOMEM = 0, 1, 2, 3, 4
 DL_GDN, DL_KDA, DL_RWKV6 = 0, 1, 2
 DL_F32, DL_BF16 = 0, 1
+DL_MERGE_OFF, DL_MERGE_FOLD, DL_MERGE_SEPARATE = 0, 1, 2
 
 # Every symbol include/deltalog.h declares.
 EXPORTS = (

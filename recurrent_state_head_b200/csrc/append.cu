@@ -1,35 +1,41 @@
-// append.cu -- launchers of the append + read-out kernel (all ops and shapes).
+// append.cu -- launchers of the append + read-out kernel and its merge-token
+// variant (all ops and shapes).
+#include <mutex>
+
 #include "launch.h"
 
 namespace dl {
 namespace {
-template <int OP, int DK, int DV, int TV>
-cudaError_t launch_tv(AppendParams p, cudaStream_t s, int sms) {
+template <int OP, int DK, int DV, int TV, bool FOLD>
+cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = 4 * TV;
-    static PlanCache cache;
-    auto kern = append_kernel<OP, DK, DV, TV, NT>;
+    static std::atomic<unsigned long long> smem_ok{0};
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD>;
     const int ie = p.in_bf16 ? 2 : 4;
-    Plan plan;
-    cudaError_t e = cache.get(kern, NT, stage_layout<OP, DK, TV>(p.L, ie, true).bytes, &plan);
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
     if (e != cudaSuccess) return e;
-    p.ns = plan.ns;
-    const long long units = (long long)p.NH * (DV / TV);
-    const int grid = (int)std::min<long long>(units, (long long)sms * plan.per_sm);
-    kern<<<grid, NT, plan.smem, s>>>(p);
+    const unsigned grid = (unsigned)p.NH * (DV / TV);
+    kern<<<grid, NT, smem, s>>>(p);
     return cudaGetLastError();
 }
 
-template <int OP, int DK, int DV>
-cudaError_t launch(const AppendParams &p, cudaStream_t s) {
-    DeviceFacts f;
-    cudaError_t e = device_facts(&f);
+template <int OP, int DK, int DV, bool FOLD>
+cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
-    switch (pick_tile(p.NH, DV, f.sms)) {
-        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128>(p, s, f.sms); break;
-        case 64: return launch_tv<OP, DK, DV, 64>(p, s, f.sms);
+    switch (pick_tile(p.NH, DV, sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, FOLD>(p, s); break;
+        case 64: return launch_tv<OP, DK, DV, 64, FOLD>(p, s);
         default: break;
     }
-    return launch_tv<OP, DK, DV, 32>(p, s, f.sms);
+    return launch_tv<OP, DK, DV, 32, FOLD>(p, s);
+}
+
+template <int OP, int DK, int DV>
+cudaError_t launch(const AppendParams &p, bool fold, cudaStream_t s) {
+    return fold ? launch_fold<OP, DK, DV, true>(p, s) : launch_fold<OP, DK, DV, false>(p, s);
 }
 
 #define ROW(OP) {{launch<OP, 64, 64>, launch<OP, 64, 128>}, {launch<OP, 128, 64>, launch<OP, 128, 128>}}
@@ -43,24 +49,19 @@ append_fn get_append(int op, int dk, int dv) {
     return table[op][a][b];
 }
 
-cudaError_t device_facts(DeviceFacts *f) {
+cudaError_t sm_count(int *sms) {
     static std::mutex mu;
-    static DeviceFacts cache[64];
+    static int cache[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (cache[dev].sms == 0) {
-        DeviceFacts d;
-        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-            return e;
-        if ((e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
-            cudaSuccess)
-            return e;
-        cache[dev] = d;
+    if (cache[dev] == 0) {
+        e = cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
     }
-    *f = cache[dev];
+    *sms = cache[dev];
     return cudaSuccess;
 }
 }  // namespace dl

@@ -56,8 +56,8 @@ dl_status check_config(const dl_config *c, bool need_log) {
         (c->out_dtype != DL_F32 && c->out_dtype != DL_BF16))
         return fail(DL_EINVAL, "dtypes must be DL_F32 or DL_BF16");
     if (!std::isfinite(c->scale)) return fail(DL_EINVAL, "scale is not finite");
-    if (need_log && c->auto_merge != 0 && c->auto_merge != 1)
-        return fail(DL_EINVAL, "auto_merge must be 0 or 1");
+    if (need_log && (c->auto_merge < DL_MERGE_OFF || c->auto_merge > DL_MERGE_SEPARATE))
+        return fail(DL_EINVAL, "auto_merge must be 0, 1 or 2");
     return DL_OK;
 }
 
@@ -151,9 +151,11 @@ dl::MergeParams merge_params(const dl_handle *h, float *dst, int L) {
     return p;
 }
 
-cudaError_t launch_append(const dl_handle *h, const dl_step_io &io, int L, cudaStream_t s) {
+// fold: the merge-token variant (the token that completes the log writes
+// the merged state over the base instead of appending).
+cudaError_t launch_append(const dl_handle *h, const dl_step_io &io, int L, bool fold, cudaStream_t s) {
     if (h->NH == 0) return cudaSuccess;
-    return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(append_params(h, io, L), s);
+    return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(append_params(h, io, L), fold, s);
 }
 
 cudaError_t launch_merge(const dl_handle *h, float *dst, int L, cudaStream_t s) {
@@ -218,10 +220,18 @@ dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void 
         return fail(DL_ESTATE, "log is full (L = C = %d) and auto_merge is off: merge first", h->cfg.C);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const dl_step_io io = {q, k, v, beta, g, out};
-    cudaError_t e = launch_append(h, io, h->L, st);
+    if (h->cfg.auto_merge == DL_MERGE_FOLD && h->L == h->cfg.C - 1) {
+        // the token that completes the log: one kernel reads the base once
+        // and writes the merged logical state back
+        cudaError_t e = launch_append(h, io, h->L, true, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge-token kernel launch");
+        h->L = 0;
+        return ok();
+    }
+    cudaError_t e = launch_append(h, io, h->L, false, st);
     if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
     h->L += 1;
-    if (h->cfg.auto_merge && h->L == h->cfg.C) {
+    if (h->cfg.auto_merge == DL_MERGE_SEPARATE && h->L == h->cfg.C) {
         e = launch_merge(h, h->base, h->L, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
         h->L = 0;
@@ -295,7 +305,7 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
         const dl_handle *h = layers[l];
         if (!h) return fail(DL_EINVAL, "layer %d is NULL", l);
         if (h->cfg.C != C) return fail(DL_EINVAL, "layers must share one log capacity C");
-        if (!h->cfg.auto_merge) return fail(DL_EINVAL, "layer %d has auto_merge = 0", l);
+        if (h->cfg.auto_merge == DL_MERGE_OFF) return fail(DL_EINVAL, "layer %d has auto_merge = 0", l);
         if (h->L != 0) return fail(DL_ESTATE, "layer %d has L = %d, a cycle starts at L = 0", l, h->L);
         for (int t = 0; t < C; ++t) {
             const dl_step_io &x = io[(size_t)t * n_layers + l];
@@ -325,14 +335,17 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
     e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
     cudaError_t le = cudaSuccess;
     if (e == cudaSuccess) {
-        // token-major: every layer's append for token t, then, after the
-        // C-th append of a layer, that layer's merge
+        // token-major: every layer's step for token t; the token that
+        // completes a layer's log is its merge-token (DL_MERGE_FOLD) or its
+        // append followed by its merge (DL_MERGE_SEPARATE)
         for (int t = 0; t < C && le == cudaSuccess; ++t) {
             for (int l = 0; l < n_layers && le == cudaSuccess; ++l) {
                 const dl_handle *h = layers[l];
-                le = launch_append(h, io[(size_t)t * n_layers + l], t, st);
+                const bool last = t == C - 1;
+                const bool fold = last && h->cfg.auto_merge == DL_MERGE_FOLD;
+                le = launch_append(h, io[(size_t)t * n_layers + l], t, fold, st);
                 if (h->NH > 0) cy->kernels += 1;
-                if (le == cudaSuccess && t == C - 1) {
+                if (le == cudaSuccess && last && h->cfg.auto_merge == DL_MERGE_SEPARATE) {
                     le = launch_merge(h, h->base, C, st);
                     if (h->NH > 0) cy->kernels += 1;
                 }

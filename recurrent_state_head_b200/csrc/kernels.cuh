@@ -11,10 +11,8 @@
 // there are too few heads to fill the GPU (the paper's value-tile split): TV
 // value columns of all d_k rows, so the key-side contractions S^T x reduce
 // inside the CTA.  NT = 4 TV threads: TV/4 threads per row, each owning a
-// 16-byte column group, 16 row groups.  The append and merge kernels are
-// persistent and stream each unit through a ring of shared-memory stages
-// filled by cp.async; the eager kernel is one CTA per 32-column tile with
-// the tile in registers.  Nothing here is a dense contraction worth a tensor
+// 16-byte column group, 16 row groups, RPT = d_k / 16 rows per thread held in
+// registers.  The eager kernel always uses 32-column tiles.  Nothing here is a dense contraction worth a tensor
 // core: per state element the append does 2 FMAs and the merge at most
 // C = 16, against 4 to 8 bytes of HBM traffic.
 #pragma once
@@ -43,7 +41,6 @@ struct AppendParams {
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
-    int ns;                   // pipeline stages (1..4)
 };
 
 struct MergeParams {
@@ -54,7 +51,6 @@ struct MergeParams {
     const float *logLam;
     int NH, C, L;
     int in_bf16;
-    int ns;                   // pipeline stages (1..4)
 };
 
 struct EagerParams {
@@ -137,15 +133,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Copy `bytes` (a multiple of 16; both addresses 16-byte aligned) with all
-// NT threads of the CTA.
-template <int NT>
-__device__ __forceinline__ void cp_async_bytes(void *smem, const void *gmem, int bytes) {
-    char *d = static_cast<char *>(smem);
-    const char *g = static_cast<const char *>(gmem);
-    for (int o = threadIdx.x * 16; o < bytes; o += NT * 16) cp_async16(d + o, g + o);
-}
-
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -201,87 +188,97 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
-// ============================================== persistent stage pipeline ==
+// ===================================================== operand staging ==
 //
-// The append and merge kernels are persistent: a grid of (SM count x
-// resident CTAs per SM) CTAs walks the units with a stride of gridDim.x.
-// Each unit's operands -- its base tile and every small operand -- form one
-// stage in dynamic shared memory, filled with cp.async.  `ns` stages rotate:
-// while unit n is computed from its stage, the copies of units n+1 .. n+ns-1
-// are in flight, so the HBM stream does not wait for a CTA's prologue,
-// reductions or epilogue.  All waits are cp.async.wait_group (hardware) and
-// __syncthreads.
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-// Wait until at most n of this thread's committed copy groups are pending.
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-    switch (n) {
-        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    }
-}
+// The append, merge-token and merge kernels hold their base tile in
+// registers (16-byte loads issued first, so they are in flight while
+// everything else happens) and stage the small operands -- the token's rows,
+// its decay, beta or bonus, and the L logged entries -- in dynamic shared
+// memory with cp.async issued by warp 0 alone, waited for with
+// cp.async.wait_all (a hardware wait) and published with __syncthreads.
 
 __host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
+__host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
-// Byte offsets of one stage (all 16-byte aligned).
-struct StageLayout {
-    int base, kin, qin, vin, g, beta, bonus, K, lam, U, bytes;
+// Byte offsets of the staged operands (all 16-byte aligned).
+struct OpLayout {
+    int kin, qin, vin, g, beta, bonus, K, lam, U, A, bytes;
 };
 
-// Append stage for log length L: base tile [DK][TV] fp32, the token's k, q
-// rows and v tile, g, beta or bonus, and the L logged entries (keys,
-// decay snapshots, the tile's value factors).  The merge stage holds the
-// base tile and the L logged entries only.
+// token: stage the token's k, q (r), v tile, g, beta / bonus.  A: room for
+// the [DK][up4(L) + 4] fp32 table of per-row replay factors (merge,
+// merge-token).
 template <int OP, int DK, int TV>
-__host__ __device__ inline StageLayout stage_layout(int L, int ie, bool append) {
+__host__ __device__ inline OpLayout op_layout(int L, int ie, bool token, bool table) {
     const int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
-    StageLayout s{};
+    OpLayout s{};
     int o = 0;
-    s.base = o; o += DK * TV * 4;
-    s.kin = o; o += append ? up16(DK * ie) : 0;
-    s.qin = o; o += append ? up16(DK * ie) : 0;
-    s.vin = o; o += append ? up16(TV * ie) : 0;
-    s.g = o; o += append ? up16(M * 4) : 0;
-    s.beta = o; o += append ? 16 : 0;
-    s.bonus = o; o += (append && OP == OP_RWKV6) ? DK * 4 : 0;
+    s.kin = o; o += token ? up16(DK * ie) : 0;
+    s.qin = o; o += token ? up16(DK * ie) : 0;
+    s.vin = o; o += token ? up16(TV * ie) : 0;
+    s.g = o; o += token ? up16(M * 4) : 0;
+    s.beta = o; o += token ? 16 : 0;
+    s.bonus = o; o += (token && OP == OP_RWKV6) ? DK * 4 : 0;
     s.K = o; o += up16(L * DK * ie);
     s.lam = o; o += up16(L * M * 4);
     s.U = o; o += up16(L * TV * ue);
+    s.A = o; o += table ? DK * (up4(L) + 4) * 4 : 0;
     s.bytes = o;
     return s;
 }
 
-// Copy a [rows][TV] fp32 tile (row stride DV floats) into shared memory.
-template <int DV, int TV, int NT>
-__device__ __forceinline__ void cp_tile(unsigned char *dst, const float *src, int rows) {
-    constexpr int CPR = TV / 4;                     // 16-byte chunks per row
-    if constexpr (TV == DV) {                       // whole rows: one contiguous block
-        cp_async_bytes<NT>(dst, src, rows * TV * 4);
-    } else {
-        for (int idx = threadIdx.x; idx < rows * CPR; idx += NT) {
-            const int r = idx / CPR, c = idx - r * CPR;
-            cp_async16(dst + (r * TV + c * 4) * 4, src + (size_t)r * DV + c * 4);
-        }
-    }
+// warp-level copy of `bytes` (a multiple of 16; 16-byte aligned addresses)
+__device__ __forceinline__ void warp_copy(unsigned char *dst, const void *src, int bytes, int lane) {
+    const char *g = static_cast<const char *>(src);
+    for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, g + o);
 }
 
-// Copy the L logged value-factor rows of one tile (row stride DV elements of
-// `ue` bytes, TV elements each) into shared memory.
-template <int DV, int TV, int NT>
-__device__ __forceinline__ void cp_logrows(unsigned char *dst, const char *src, int L, int ue) {
-    if constexpr (TV == DV) {
-        cp_async_bytes<NT>(dst, src, L * TV * ue);
-    } else {
-        const int cpr = TV * ue / 16;
-        for (int idx = threadIdx.x; idx < L * cpr; idx += NT) {
-            const int j = idx / cpr, c = idx - j * cpr;
-            cp_async16(dst + j * TV * ue + c * 16, src + (size_t)j * DV * ue + c * 16);
+// Sources of one head's staged operands.
+struct OpSources {
+    const void *k, *q, *v;          // token rows (NULL: not staged)
+    const float *g, *beta, *bonus;
+    const void *logK, *logU;
+    const float *logLam;
+};
+
+// Stage one unit's operands (warp 0 only), then wait for them.
+template <int OP, int DK, int DV, int TV>
+__device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay, const OpSources &src,
+                                          int head, int vt, int L, int C, int H, int ie, bool token) {
+    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    const int ue = (OP == OP_RWKV6) ? ie : 4;
+    const int lane = threadIdx.x & 31;
+    if (token) {
+        warp_copy(sm + lay.kin, static_cast<const char *>(src.k) + (size_t)head * DK * ie, DK * ie, lane);
+        warp_copy(sm + lay.qin, static_cast<const char *>(src.q) + (size_t)head * DK * ie, DK * ie, lane);
+        warp_copy(sm + lay.vin, static_cast<const char *>(src.v) + ((size_t)head * DV + vt * TV) * ie,
+                  TV * ie, lane);
+        if (OP == OP_GDN) {
+            if (lane == 0) cp_async4(sm + lay.g, src.g + head);
+        } else {
+            warp_copy(sm + lay.g, src.g + (size_t)head * DK, DK * 4, lane);
         }
+        if (OP == OP_RWKV6)
+            warp_copy(sm + lay.bonus, src.bonus + (size_t)(head % H) * DK, DK * 4, lane);
+        else if (lane == 1)
+            cp_async4(sm + lay.beta, src.beta + head);
     }
+    warp_copy(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie, L * DK * ie,
+              lane);
+    const float *lamh = src.logLam + (size_t)head * C * M;
+    if (OP == OP_GDN) {
+        for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
+    } else {
+        warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
+    }
+    const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
+    const int cpr = TV * ue / 16;
+    for (int idx = lane; idx < L * cpr; idx += 32) {
+        const int j = idx / cpr, c = idx - j * cpr;
+        cp_async16(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16);
+    }
+    cp_async_wait_all();
 }
 
 // Four consecutive elements of a raw vector in shared memory as fp32.
@@ -294,15 +291,63 @@ __device__ __forceinline__ float4 ld_raw4(const unsigned char *p, int i, int bf1
     return *reinterpret_cast<const float4 *>(p + 4 * i);
 }
 
-// ====================================================== append + read-out ==
+// Replay-factor table A[i][j] = exp(lam[i] - Lambda_j[i]) k_j[i] for j < L
+// (pitch up4(L) + 4 floats) and the base decay gam[i] = exp(lam[i]), where
+// lam is Lambda_L (merge) or Lambda_t (merge-token).  All NT threads.
+template <int OP, int DK, int NT>
+__device__ __forceinline__ void replay_table(float *A, float *gam, const float *lam_row,
+                                             const unsigned char *sK, const float *slam, int L, int bf16) {
+    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    const int AP = up4(L) + 4;
+    for (int idx = threadIdx.x; idx < DK * (L + 1); idx += NT) {
+        const int i = idx % DK, j = idx / DK;           // j == L -> base decay
+        const int x = (OP == OP_GDN) ? 0 : i;
+        if (j == L)
+            gam[i] = expf(lam_row[x]);
+        else
+            A[i * AP + j] = expf(lam_row[x] - slam[j * M + x]) * ld_raw(sK, j * DK + i, bf16);
+    }
+}
+
+// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3] (+ kr * w4)
+template <int TV>
+__device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow, const unsigned char *sU,
+                                           int c4, int L, int ubf) {
+    float4 o = make_float4(gm * s.x, gm * s.y, gm * s.z, gm * s.w);
+    for (int j0 = 0; j0 < L; j0 += 4) {
+        const float4 cf4 = *reinterpret_cast<const float4 *>(Arow + j0);
+        const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            if (j0 + jj < L) {
+                const float4 u = ld_raw4(sU, (j0 + jj) * TV + c4, ubf);
+                o.x = fmaf(cf[jj], u.x, o.x);
+                o.y = fmaf(cf[jj], u.y, o.y);
+                o.z = fmaf(cf[jj], u.z, o.z);
+                o.w = fmaf(cf[jj], u.w, o.w);
+            }
+        }
+    }
+    return o;
+}
+
+// ============================================ append + read-out (+ fold) ==
 //
-// ReplayPrep (once per unit, from its stage): the decay point Lambda_t
-// (RWKV6: Lambda_{t-1}), read-out weights Gamma * k and Gamma * q (RWKV6:
-// Gamma * r), replay coefficients c_j = sum_i k_i K_j[i] e^{Lam[i] - Lam_j[i]}
-// (d_j with q) and the self term.  AppendDecode: x = Sbar^T w over the tile
-// (the one base read), value-side replay, delta correction, output, append
-// of u (and, by the first tile of each head, of k and Lambda_t).
-template <int OP, int DK, int DV, int TV, int NT>
+// One CTA per unit (a head, or a TV-column value tile of a head).
+// ReplayPrep (once per CTA): decay point Lambda_t = Lambda_{L-1} + g_t
+// (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
+// Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
+// (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
+// x = Sbar^T w over the register tile (the one base read), value-side replay,
+// delta correction, output.
+// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
+//   slot L; the base is not written.
+// FOLD = true (merge-token, the step that completes the log: "Fase di
+//   Merge"): the logical state after this token -- base decayed to Lambda_t,
+//   all L logged factors and this token's k u^T -- is written over the base
+//   tile (the register tile is read once and written once); the log is left
+//   for the caller to reset (L = 0).
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
@@ -311,189 +356,184 @@ append_kernel(const AppendParams p) {
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
     extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ float s_lt[DK];           // Lambda_t
     __shared__ float s_lr[DK];           // decay point of read-out and replay
     __shared__ float s_k[DK];
     __shared__ float s_q[DK];
     __shared__ float s_w[NA][DK];        // read-out weights
     __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
+    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
+    __shared__ __align__(16) float s_red[NA * T::NW * TV];
     __shared__ float s_x[NA * TV];
-    static_assert(NA * T::NW * TV <= DK * TV, "row partials fit in the consumed base tile");
+    __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
+    const int unit = blockIdx.x;
+    const int head = unit / T::NVT, vt = unit - head * T::NVT;
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C, ns = p.ns;
+    const int L = p.L, C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
-    const int ue = (OP == OP_RWKV6) ? ie : 4;
-    const StageLayout lay = stage_layout<OP, DK, TV>(L, ie, true);
-    const int n_units = p.NH * T::NVT;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
+    const int c4 = col4 * 4;
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
 
-    auto issue = [&](int unit, unsigned char *st) {
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        cp_tile<DV, TV, NT>(st + lay.base, p.base + (size_t)head * DK * DV + vt * TV, DK);
-        cp_async_bytes<NT>(st + lay.kin, static_cast<const char *>(p.k) + (size_t)head * DK * ie, DK * ie);
-        cp_async_bytes<NT>(st + lay.qin, static_cast<const char *>(p.q) + (size_t)head * DK * ie, DK * ie);
-        cp_async_bytes<NT>(st + lay.vin,
-                           static_cast<const char *>(p.v) + ((size_t)head * DV + vt * TV) * ie, TV * ie);
-        cp_async_bytes<NT>(st + lay.K, static_cast<const char *>(p.logK) + (size_t)head * C * DK * ie,
-                           L * DK * ie);
-        const float *lamh = p.logLam + (size_t)head * C * M;
-        if (OP == OP_GDN) {
-            if (tid == 0) cp_async4(st + lay.g, p.g + head);
-            for (int j = tid; j < L; j += NT) cp_async4(st + lay.lam + 4 * j, lamh + j);
+    // 1. the base stream: RPT rows x 16 bytes per thread
+    float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
+                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+
+    // 2. small operands, staged by warp 0 while the base loads are in flight
+    if (tid < 32) {
+        const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true);
+    }
+    __syncthreads();
+    const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
+
+    // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
+    if (tid < DK) {
+        const int i = tid;
+        const int x = (OP == OP_GDN) ? 0 : i;
+        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+        const float lt = lprev + sg[x];
+        const float lr = (OP == OP_RWKV6) ? lprev : lt;
+        const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
+        const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
+        const float gam = expf(lr);
+        s_lt[i] = lt;
+        s_lr[i] = lr;
+        s_k[i] = kf;
+        s_q[i] = qf;
+        if (OP == OP_RWKV6) {
+            s_w[0][i] = gam * qf;
+            s_bk[i] = reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf;
         } else {
-            cp_async_bytes<NT>(st + lay.g, p.g + (size_t)head * DK, DK * 4);
-            cp_async_bytes<NT>(st + lay.lam, lamh, L * DK * 4);
+            s_w[0][i] = gam * kf;
+            s_w[NA - 1][i] = gam * qf;
         }
-        if (OP == OP_RWKV6)
-            cp_async_bytes<NT>(st + lay.bonus, p.bonus + (size_t)(head % p.H) * DK, DK * 4);
-        else if (tid == NT - 1)
-            cp_async4(st + lay.beta, p.beta + head);
-        cp_logrows<DV, TV, NT>(st + lay.U,
-                               static_cast<const char *>(p.logU) + ((size_t)head * C * DV + vt * TV) * ue,
-                               L, ue);
-    };
+        if (!FOLD && vt == 0) {
+            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
+            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
+        }
+    }
+    __syncthreads();
 
-    for (int s = 0; s < ns - 1; ++s) {
-        const int u = blockIdx.x + s * gridDim.x;
-        if (u < n_units) issue(u, dsm + s * lay.bytes);
-        cp_async_commit();
+    // replay coefficients: task tau < L is log entry tau, tau == L the self term
+    {
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int tau = warp; tau <= L; tau += T::NW) {
+            float a0 = 0.f, a1 = 0.f;
+            if (tau < L) {
+                const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
+#pragma unroll
+                for (int i = lane; i < DK; i += 32) {
+                    const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
+                    const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
+                    if (OP == OP_RWKV6) {
+                        a0 = fmaf(s_q[i], e, a0);
+                    } else {
+                        a0 = fmaf(s_k[i], e, a0);
+                        a1 = fmaf(s_q[i], e, a1);
+                    }
+                }
+                a0 = warp_sum(a0) * gdec;
+                if (NA == 2) a1 = warp_sum(a1) * gdec;
+                if (lane == 0) {
+                    s_coef[0][tau] = a0;
+                    if (NA == 2) s_coef[NA - 1][tau] = a1;
+                }
+            } else {
+#pragma unroll
+                for (int i = lane; i < DK; i += 32)
+                    a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
+                a0 = warp_sum(a0);
+                if (lane == 0) s_self = a0;
+            }
+        }
+    }
+    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
+                                       dsm + lay.K, slam, L, p.in_bf16);
+    __syncthreads();
+
+    // 4. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    {
+        float4 acc[NA];
+#pragma unroll
+        for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+#pragma unroll
+            for (int a = 0; a < NA; ++a) {
+                const float w = s_w[a][row];
+                acc[a].x = fmaf(w, s[r].x, acc[a].x);
+                acc[a].y = fmaf(w, s[r].y, acc[a].y);
+                acc[a].z = fmaf(w, s[r].z, acc[a].z);
+                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+            }
+        }
+        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
     }
 
-    for (int it = 0;; ++it) {
-        const int unit = blockIdx.x + it * gridDim.x;
-        if (unit >= n_units) break;
-        {
-            const int un = unit + (ns - 1) * gridDim.x;
-            if (un < n_units) issue(un, dsm + ((it + ns - 1) % ns) * lay.bytes);
-            cp_async_commit();
-        }
-        cp_async_wait_pending(ns - 1);
-        __syncthreads();
-
-        const unsigned char *st = dsm + (it % ns) * lay.bytes;
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        const float *sg = reinterpret_cast<const float *>(st + lay.g);
-        const float *slam = reinterpret_cast<const float *>(st + lay.lam);
-
-        // key side: decay point, read-out weights, append of k and Lambda_t
-        if (tid < DK) {
-            const int i = tid;
-            const int x = (OP == OP_GDN) ? 0 : i;
-            const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-            const float lt = lprev + sg[x];
-            const float lr = (OP == OP_RWKV6) ? lprev : lt;
-            const float kf = ld_raw(st + lay.kin, i, p.in_bf16);
-            const float qf = ld_raw(st + lay.qin, i, p.in_bf16);
-            const float gam = expf(lr);
-            s_lr[i] = lr;
-            s_k[i] = kf;
-            s_q[i] = qf;
-            if (OP == OP_RWKV6) {
-                s_w[0][i] = gam * qf;
-                s_bk[i] = reinterpret_cast<const float *>(st + lay.bonus)[i] * kf;
-            } else {
-                s_w[0][i] = gam * kf;
-                s_w[NA - 1][i] = gam * qf;
+    // 5. value side: log replay, delta correction, output, append of u
+    if (tid < TV) {
+        const int c = tid;
+        const int col = vt * TV + c;
+        const size_t ub = (size_t)head * C * DV + col;
+        const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
+        if (OP == OP_RWKV6) {
+            float rr = 0.f;
+            for (int j = 0; j < L; ++j)
+                rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
+            const float o = p.scale * (s_x[c] + rr + s_self * vv);
+            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+            if (FOLD)
+                s_u[c] = vv;
+            else
+                copy_raw(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16);
+        } else {
+            const float *U = reinterpret_cast<const float *>(dsm + lay.U);
+            float rk = 0.f, rq = 0.f;
+            for (int j = 0; j < L; ++j) {
+                const float uj = U[j * TV + c];
+                rk = fmaf(s_coef[0][j], uj, rk);
+                rq = fmaf(s_coef[1][j], uj, rq);
             }
-            if (vt == 0) {
-                copy_raw(p.logK, ((size_t)head * C + L) * DK + i, st + lay.kin, i, p.in_bf16);
-                if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
-            }
-        }
-        __syncthreads();
-
-        // replay coefficients: task tau < L is log entry tau, tau == L the self term
-        {
-            const int lane = tid & 31, warp = tid >> 5;
-            for (int tau = warp; tau <= L; tau += T::NW) {
-                float a0 = 0.f, a1 = 0.f;
-                if (tau < L) {
-                    const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
-#pragma unroll
-                    for (int i = lane; i < DK; i += 32) {
-                        const float kj = ld_raw(st + lay.K, tau * DK + i, p.in_bf16);
-                        const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
-                        if (OP == OP_RWKV6) {
-                            a0 = fmaf(s_q[i], e, a0);
-                        } else {
-                            a0 = fmaf(s_k[i], e, a0);
-                            a1 = fmaf(s_q[i], e, a1);
-                        }
-                    }
-                    a0 = warp_sum(a0) * gdec;
-                    if (NA == 2) a1 = warp_sum(a1) * gdec;
-                    if (lane == 0) {
-                        s_coef[0][tau] = a0;
-                        if (NA == 2) s_coef[NA - 1][tau] = a1;
-                    }
-                } else {
-#pragma unroll
-                    for (int i = lane; i < DK; i += 32)
-                        a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
-                    a0 = warp_sum(a0);
-                    if (lane == 0) s_self = a0;
-                }
-            }
-        }
-        __syncthreads();
-
-        // base read-out from the staged tile: x_a[c] = sum_i w_a[i] * Sbar[i][c];
-        // the row partials are then reduced through the consumed tile
-        {
-            float *tile = reinterpret_cast<float *>(dsm + (it % ns) * lay.bytes + lay.base);
-            float4 acc[NA];
-#pragma unroll
-            for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const int row = rg + r * T::RG;
-                const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + col4 * 4);
-#pragma unroll
-                for (int a = 0; a < NA; ++a) {
-                    const float w = s_w[a][row];
-                    acc[a].x = fmaf(w, sv.x, acc[a].x);
-                    acc[a].y = fmaf(w, sv.y, acc[a].y);
-                    acc[a].z = fmaf(w, sv.z, acc[a].z);
-                    acc[a].w = fmaf(w, sv.w, acc[a].w);
-                }
-            }
-            __syncthreads();
-            reduce_rows<NA, TV, NT>(acc, tile, s_x);
-        }
-
-        // value side: log replay, delta correction, output, append of u
-        if (tid < TV) {
-            const int c = tid;
-            const int col = vt * TV + c;
-            const size_t ub = (size_t)head * C * DV + col;
-            const float vv = ld_raw(st + lay.vin, c, p.in_bf16);
-            if (OP == OP_RWKV6) {
-                float rr = 0.f;
-                for (int j = 0; j < L; ++j)
-                    rr = fmaf(s_coef[0][j], ld_raw(st + lay.U, j * TV + c, p.in_bf16), rr);
-                const float o = p.scale * (s_x[c] + rr + s_self * vv);
-                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-                copy_raw(p.logU, ub + (size_t)L * DV, st + lay.vin, c, p.in_bf16);
-            } else {
-                const float *U = reinterpret_cast<const float *>(st + lay.U);
-                float rk = 0.f, rq = 0.f;
-                for (int j = 0; j < L; ++j) {
-                    const float uj = U[j * TV + c];
-                    rk = fmaf(s_coef[0][j], uj, rk);
-                    rq = fmaf(s_coef[1][j], uj, rq);
-                }
-                const float beta = *reinterpret_cast<const float *>(st + lay.beta);
-                const float u = beta * (vv - s_x[c] - rk);
-                const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
-                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+            const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
+            const float u = beta * (vv - s_x[c] - rk);
+            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+            if (FOLD)
+                s_u[c] = u;
+            else
                 reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
-            }
         }
-        __syncthreads();   // the stage is refilled by a later iteration's copies
     }
-    cp_async_wait_pending(0);
+
+    // 6. merge-token: write the logical state after this token over the base
+    if (FOLD) {
+        __syncthreads();
+        const float *A = reinterpret_cast<const float *>(dsm + lay.A);
+        const int AP = up4(L) + 4;
+        const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+        const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+            const float kr = s_k[row];
+            o.x = fmaf(kr, u4.x, o.x);
+            o.y = fmaf(kr, u4.y, o.y);
+            o.z = fmaf(kr, u4.z, o.z);
+            o.w = fmaf(kr, u4.w, o.w);
+            st_state(bh + (size_t)row * DV, o);
+        }
+    }
 }
 
 // ================================================= merge / materialise ==
@@ -501,103 +541,53 @@ append_kernel(const AppendParams p) {
 // dst[i][c] = exp(Lambda_L[i]) base[i][c] + sum_{j<L} exp(Lambda_L[i] - Lambda_j[i]) k_j[i] u_j[c]
 // (Lambda_L = the last entry's snapshot; L = 0 copies the base).  In place
 // (dst == base) it is the merge; into another buffer it is materialise.
-// Persistent, with the same stage pipeline as the append kernel.
+// One CTA per unit; the register tile is loaded first, the log staged by
+// warp 0, the replay-factor table built once per CTA.
 template <int OP, int DK, int DV, int TV, int NT>
 __global__ void __launch_bounds__(NT)
 merge_kernel(const MergeParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
-    constexpr int CP = MAXC + 4;             // row pitch of the coefficient table
 
     extern __shared__ __align__(16) unsigned char dsm[];
     __shared__ float s_gam[DK];
-    __shared__ __align__(16) float s_coef[DK * CP];   // [row][entry]
+    __shared__ float s_lL[M];
 
+    const int unit = blockIdx.x;
+    const int head = unit / T::NVT, vt = unit - head * T::NVT;
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C, ns = p.ns;
+    const int L = p.L, C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
-    const int ue = (OP == OP_RWKV6) ? ie : 4;
-    const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-    const StageLayout lay = stage_layout<OP, DK, TV>(L, ie, false);
-    const int n_units = p.NH * T::NVT;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
+    const int c4 = col4 * 4;
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, false, true);
 
-    auto issue = [&](int unit, unsigned char *st) {
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        cp_tile<DV, TV, NT>(st + lay.base, p.base + (size_t)head * DK * DV + vt * TV, DK);
-        cp_async_bytes<NT>(st + lay.K, static_cast<const char *>(p.logK) + (size_t)head * C * DK * ie,
-                           L * DK * ie);
-        const float *lamh = p.logLam + (size_t)head * C * M;
-        if (OP == OP_GDN) {
-            for (int j = tid; j < L; j += NT) cp_async4(st + lay.lam + 4 * j, lamh + j);
-        } else {
-            cp_async_bytes<NT>(st + lay.lam, lamh, L * DK * 4);
-        }
-        cp_logrows<DV, TV, NT>(st + lay.U,
-                               static_cast<const char *>(p.logU) + ((size_t)head * C * DV + vt * TV) * ue,
-                               L, ue);
-    };
-
-    for (int s = 0; s < ns - 1; ++s) {
-        const int u = blockIdx.x + s * gridDim.x;
-        if (u < n_units) issue(u, dsm + s * lay.bytes);
-        cp_async_commit();
-    }
-
-    for (int it = 0;; ++it) {
-        const int unit = blockIdx.x + it * gridDim.x;
-        if (unit >= n_units) break;
-        {
-            const int un = unit + (ns - 1) * gridDim.x;
-            if (un < n_units) issue(un, dsm + ((it + ns - 1) % ns) * lay.bytes);
-            cp_async_commit();
-        }
-        cp_async_wait_pending(ns - 1);
-        __syncthreads();
-
-        const unsigned char *st = dsm + (it % ns) * lay.bytes;
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        const float *slam = reinterpret_cast<const float *>(st + lay.lam);
-
-        // per-row decay of the base and replay coefficients
-        for (int idx = tid; idx < DK * (L + 1); idx += NT) {
-            const int i = idx % DK, j = idx / DK;          // j == L -> base decay
-            const int x = (OP == OP_GDN) ? 0 : i;
-            const float lL = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-            if (j == L)
-                s_gam[i] = expf(lL);
-            else
-                s_coef[i * CP + j] = expf(lL - slam[j * M + x]) * ld_raw(st + lay.K, j * DK + i, p.in_bf16);
-        }
-        __syncthreads();
-
-        const float *tile = reinterpret_cast<const float *>(st + lay.base);
-        float *dh = p.dst + (size_t)head * DK * DV + vt * TV + col4 * 4;
-#pragma unroll 2
-        for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            const float gm = s_gam[row];
-            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + col4 * 4);
-            float4 o = make_float4(gm * sv.x, gm * sv.y, gm * sv.z, gm * sv.w);
-            for (int j0 = 0; j0 < L; j0 += 4) {
-                const float4 cf4 = *reinterpret_cast<const float4 *>(&s_coef[row * CP + j0]);
-                const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+    const float *bh = p.base + (size_t)head * DK * DV + vt * TV + c4;
+    float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    if (j0 + jj < L) {
-                        const float4 u = ld_raw4(st + lay.U, (j0 + jj) * TV + col4 * 4, ubf);
-                        o.x = fmaf(cf[jj], u.x, o.x);
-                        o.y = fmaf(cf[jj], u.y, o.y);
-                        o.z = fmaf(cf[jj], u.z, o.z);
-                        o.w = fmaf(cf[jj], u.w, o.w);
-                    }
-                }
-            }
-            st_state(dh + (size_t)row * DV, o);
-        }
-        __syncthreads();   // the stage is refilled by a later iteration's copies
+    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
+
+    if (tid < 32) {
+        const OpSources src{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false);
     }
-    cp_async_wait_pending(0);
+    __syncthreads();
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
+    for (int x = tid; x < M; x += NT) s_lL[x] = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+    __syncthreads();
+    replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lL, dsm + lay.K, slam, L,
+                             p.in_bf16);
+    __syncthreads();
+
+    const float *A = reinterpret_cast<const float *>(dsm + lay.A);
+    const int AP = up4(L) + 4;
+    const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) {
+        const int row = rg + r * T::RG;
+        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+    }
 }
 
 // ================================================================ eager ==

@@ -4,32 +4,30 @@
 namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV>
-cudaError_t launch_tv(MergeParams p, cudaStream_t s, int sms) {
+cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
     constexpr int NT = 4 * TV;
-    static PlanCache cache;
+    static std::atomic<unsigned long long> smem_ok{0};
     auto kern = merge_kernel<OP, DK, DV, TV, NT>;
     const int ie = p.in_bf16 ? 2 : 4;
-    Plan plan;
-    cudaError_t e = cache.get(kern, NT, stage_layout<OP, DK, TV>(p.L, ie, false).bytes, &plan);
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, true).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, true).bytes);
     if (e != cudaSuccess) return e;
-    p.ns = plan.ns;
-    const long long units = (long long)p.NH * (DV / TV);
-    const int grid = (int)std::min<long long>(units, (long long)sms * plan.per_sm);
-    kern<<<grid, NT, plan.smem, s>>>(p);
+    const unsigned grid = (unsigned)p.NH * (DV / TV);
+    kern<<<grid, NT, smem, s>>>(p);
     return cudaGetLastError();
 }
 
 template <int OP, int DK, int DV>
 cudaError_t launch(const MergeParams &p, cudaStream_t s) {
-    DeviceFacts f;
-    cudaError_t e = device_facts(&f);
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
-    switch (pick_tile(p.NH, DV, f.sms)) {
-        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128>(p, s, f.sms); break;
-        case 64: return launch_tv<OP, DK, DV, 64>(p, s, f.sms);
+    switch (pick_tile(p.NH, DV, sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128>(p, s); break;
+        case 64: return launch_tv<OP, DK, DV, 64>(p, s);
         default: break;
     }
-    return launch_tv<OP, DK, DV, 32>(p, s, f.sms);
+    return launch_tv<OP, DK, DV, 32>(p, s);
 }
 
 #define ROW(OP) {{launch<OP, 64, 64>, launch<OP, 64, 128>}, {launch<OP, 128, 64>, launch<OP, 128, 128>}}

@@ -48,7 +48,8 @@ def cfg(**kw):
 @pytest.mark.parametrize("bad", [
     dict(op=3), dict(op=-1), dict(B=-1), dict(H=0), dict(dk=32), dict(dv=96),
     dict(dk=256), dict(C=0), dict(C=17), dict(in_dtype=2), dict(out_dtype=-1),
-    dict(scale=float("nan")), dict(scale=float("inf")), dict(auto_merge=2),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(auto_merge=3),
+    dict(auto_merge=-1),
 ])
 def test_invalid_configs_rejected(lib, bad):
     c = cfg(**bad)
@@ -135,7 +136,8 @@ def test_failed_launch_is_reported_and_leaves_handle(lib):
 
 
 @pytest.mark.parametrize("C", [1, 2, 3, 5, 16])
-def test_schedule_matches_oracle_without_heads(lib, C, oracle_lib):
+@pytest.mark.parametrize("mode", [B.DL_MERGE_FOLD, B.DL_MERGE_SEPARATE])
+def test_schedule_matches_oracle_without_heads(lib, C, mode, oracle_lib):
     """B = 0: nothing is launched, but L advances exactly as the oracle's
     schedule (append; merge when L reaches C)."""
     import oracle
@@ -143,7 +145,7 @@ def test_schedule_matches_oracle_without_heads(lib, C, oracle_lib):
     st = oracle.LogState(oracle.GDN, np.zeros((0, 2, 2)), C)
     z = np.zeros((T, 0, 2))
     _, Ltr, merged = oracle.deltalog_run(st, z, z, z, np.zeros((T, 0)), np.zeros((T, 0, 1)))
-    hh = B.dl_create(cfg(B=0, C=C), None, None, None)
+    hh = B.dl_create(cfg(B=0, C=C, auto_merge=mode), None, None, None)
     try:
         got = []
         for t in range(T):

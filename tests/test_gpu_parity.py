@@ -104,19 +104,24 @@ def run_deltalog(w, x, S0, bonus, C, check_every_step=None, auto_merge=1):
     return layer, outs, Ls, mats
 
 
+MODES = (B.DL_MERGE_FOLD, B.DL_MERGE_SEPARATE)
+
+
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims", SHAPES)
 @pytest.mark.parametrize("C", [1, 2, 3, 4, 8, 16])
-def test_deltalog_matches_eager_oracle(op, dims, C):
+@pytest.mark.parametrize("mode", MODES)
+def test_deltalog_matches_eager_oracle(op, dims, C, mode):
     """Outputs every token, the logical (materialised) state after every
     token and the log-length schedule, over two full cycles and a ragged
-    third."""
+    third, with the merge folded into the C-th token or run separately."""
     w = small(op, *dims, C=C, T=2 * C + 3, seed=11 + C)
     S0 = synth.initial_state(w)
     bonus = synth.bonus(w)
     ti = synth.tokens(w, 0, w.T)
     x = D.to_device(ti, w)
-    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True,
+                                         auto_merge=mode)
     Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
     st = oracle.LogState(w.op, Sr, C)
     _, L_ref, _ = oracle.deltalog_run(st, q, k, v, None if op == synth.RWKV6 else beta, g, bon,
@@ -135,19 +140,22 @@ def test_deltalog_matches_eager_oracle(op, dims, C):
 
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims", SHAPES)
-@pytest.mark.parametrize("nh", [200, 300])
-def test_deltalog_tile_widths(op, dims, nh):
-    """Head counts that select each unit width of the persistent kernels (a
-    whole head per unit from two units per SM up, halved value tiles below;
-    on a 148-SM B200: 300 heads -> whole heads, 200 -> 64 columns for
-    d_v = 128).  Every head, every token, and the logical state each token."""
+@pytest.mark.parametrize("nh", [300, 600])
+@pytest.mark.parametrize("mode", MODES)
+def test_deltalog_tile_widths(op, dims, nh, mode):
+    """Head counts that select each value-tile width (a whole head per CTA
+    while that gives four CTAs per SM, halved tiles below; on a 148-SM B200:
+    600 heads -> whole heads, 300 -> 64 columns for d_v = 128, 15 heads in
+    the other tests -> 32 columns).  Every head, every token, and the logical
+    state after each token."""
     C = 4
     w = small(op, *dims, C=C, T=2 * C + 3, Bsz=nh // 4, H=4, seed=40 + nh)
     S0 = synth.initial_state(w)
     bonus = synth.bonus(w)
     ti = synth.tokens(w, 0, w.T)
     x = D.to_device(ti, w)
-    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True,
+                                         auto_merge=mode)
     Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
     o = to_np(outs)
     S = Sr
@@ -207,13 +215,14 @@ def test_log_contents(op, in_dt):
 
 
 @pytest.mark.parametrize("op", OPS)
-def test_capacity_one_equals_gpu_eager(op):
+@pytest.mark.parametrize("mode", MODES)
+def test_capacity_one_equals_gpu_eager(op, mode):
     w = small(op, 128, 128, C=1, T=9)
     S0 = synth.initial_state(w)
     bonus = synth.bonus(w)
     ti = synth.tokens(w, 0, w.T)
     x = D.to_device(ti, w)
-    layer, outs, Ls, _ = run_deltalog(w, x, S0, bonus, 1)
+    layer, outs, Ls, _ = run_deltalog(w, x, S0, bonus, 1, auto_merge=mode)
     assert Ls == [0] * w.T
     S = torch.from_numpy(S0).reshape(w.heads, w.dk, w.dv).cuda()
     bon_d = None if bonus is None else torch.from_numpy(bonus).cuda()
@@ -269,7 +278,8 @@ def test_explicit_merge_and_materialize(op):
 
 
 @pytest.mark.parametrize("op", OPS)
-def test_cycle_graph_equals_steps(op):
+@pytest.mark.parametrize("mode", MODES)
+def test_cycle_graph_equals_steps(op, mode):
     """One graph-captured merge cycle over two layers gives the same bytes as
     the same steps issued one by one."""
     C = 4
@@ -279,8 +289,8 @@ def test_cycle_graph_equals_steps(op):
         S0 = synth.initial_state(w, layer=l)
         bonus = synth.bonus(w, layer=l)
         xs.append(D.to_device(synth.tokens(w, 0, C, layer=l), w))
-        layers_a.append(D.DecodeLayer(w, S0, bonus))
-        layers_b.append(D.DecodeLayer(w, S0, bonus))
+        layers_a.append(D.DecodeLayer(w, S0, bonus, auto_merge=mode))
+        layers_b.append(D.DecodeLayer(w, S0, bonus, auto_merge=mode))
     outs_a = [layers_a[l].new_out(C) for l in range(2)]
     outs_b = [layers_b[l].new_out(C) for l in range(2)]
     for t in range(C):
@@ -290,7 +300,7 @@ def test_cycle_graph_equals_steps(op):
              None if op == synth.RWKV6 else xs[l]["beta"][t], xs[l]["g"][t], outs_b[l][t])
             for l in range(2)] for t in range(C)]
     cyc = B.Cycle([lb.handle for lb in layers_b], ios)
-    assert cyc.kernels == 2 * (C + 1)
+    assert cyc.kernels == 2 * (C + 1 if mode == B.DL_MERGE_SEPARATE else C)
     cyc.launch()
     torch.cuda.synchronize()
     for l in range(2):
@@ -310,7 +320,7 @@ def test_no_heads_on_gpu():
 
 # ------------------------------------------------ full-size workloads ----
 
-def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123):
+def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123, mode=B.DL_MERGE_FOLD):
     T = w.T if T is None else T
     rng = np.random.default_rng(seed)
     heads = np.unique(np.concatenate([[0, w.heads - 1],
@@ -320,7 +330,7 @@ def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123):
         bonus = synth.bonus(w, layer=l)
         ti = synth.tokens(w, 0, T, layer=l, want64=False)
         x = D.to_device(ti, w)
-        layer = D.DecodeLayer(w, S0, bonus)
+        layer = D.DecodeLayer(w, S0, bonus, auto_merge=mode)
         outs = layer.new_out(T)
         for t in range(T):
             layer.step(x, t, outs[t])
@@ -357,8 +367,9 @@ def test_full_gdn_fp32_small():
 @pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c4",
                                   "kda-b128-h32-d128-c8", "rwkv6-b128-h32-d64-c4",
                                   "rwkv6-b128-h32-d64-c8"])
-def test_full_size_256_tokens(name):
-    _full_size_check(synth.WORKLOADS[name])
+@pytest.mark.parametrize("mode", MODES)
+def test_full_size_256_tokens(name, mode):
+    _full_size_check(synth.WORKLOADS[name], mode=mode)
 
 
 @pytest.mark.parametrize("C", [1, 2, 16])

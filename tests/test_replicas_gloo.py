@@ -53,11 +53,16 @@ def test_single_rank_identity():
 
 def test_bytes_model_matches_hand_count():
     """Per-head bytes of the GDN B128 H16 d128 C8 workload: state 64 KiB,
-    log entry 772 B, inputs 776 B, output 256 B; amortised per token
-    77 978 B read and 9 220 B written."""
+    log entry 772 B, inputs 776 B, output 256 B.  Amortised per token:
+    with a separate merge 77 978 B read and 9 220 B written; with the
+    merge-token (7 appends + one step that reads and writes the base)
+    552 112 / 8 = 69 014 B read and 72 988 / 8 = 9 123.5 B written."""
     import bench
     from recurrent_state_head_b200 import synth
-    bm = bench.bytes_model(synth.WORKLOADS["gdn-b128-h16-d128-c8"])
+    w = synth.WORKLOADS["gdn-b128-h16-d128-c8"]
+    bm = bench.bytes_model(w, fold=False)
     assert (bm["S"], bm["E"], bm["I"], bm["O"]) == (65536, 772, 776, 256)
     assert bm["token_read"] == 77978 and bm["token_write"] == 9220
     assert bm["eager"] == (65536 + 776, 65536 + 256)
+    bf = bench.bytes_model(w, fold=True)
+    assert bf["token_read"] == 69014 and bf["token_write"] == 9123.5
