@@ -290,56 +290,58 @@ def _time_graph(launch, stream, steps, warmup, dev):
     return e0.elapsed_time(e1)
 
 
-def kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps, merge_layers=None):
+def kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps, prime, merge_layers=None):
     """Per-launch device time of every kernel of a merge cycle, from CUDA
-    timing events captured between the kernels of a graph (external event
-    nodes) and replayed `reps` times on the launching stream.
+    timing events recorded on the launching stream between kernels.
 
-    layers: decode layers in one automatic merge mode (each dl_decode_step is
-    one kernel in DL_MERGE_FOLD).  merge_layers (optional): layers with
-    auto_merge off, for the separate merge kernel (dl_merge)."""
+    The kernels are launched through the C ABI with pointers prepared in
+    advance, right after `prime()` (one cycle-graph launch) has queued a
+    millisecond of GPU work, so that the host stays ahead of the GPU and the
+    events bracket kernel time only.  layers: decode layers in merge-token
+    mode (each dl_decode_step is one kernel); merge_layers (optional): layers
+    with auto_merge off, for the separate merge kernel (dl_merge)."""
+    import ctypes
     import torch
     from recurrent_state_head_b200 import binding as B
-    recs = []
-    g = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(stream)
-    fold = layers[0].cfg.auto_merge == B.DL_MERGE_FOLD
+    lib = B.lib()
+    st = stream.cuda_stream
 
-    def ev():
-        e = torch.cuda.Event(enable_timing=True, external=True)
-        e.record(side)
-        return e
+    def io(t, l):
+        x = xs[l]
+        return (x["q"][t].data_ptr(), x["k"][t].data_ptr(), x["v"][t].data_ptr(),
+                None if w.op == 2 else x["beta"][t].data_ptr(), x["g"][t].data_ptr(),
+                outs[l][t].data_ptr())
 
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(g, stream=side):
-            prev = ev()
-            for t in range(C):
-                for l in range(R):
-                    layers[l].step(xs[l], t, outs[l][t], side)
-                    e = ev()
-                    recs.append(("merge_token" if fold and t == C - 1 else "append", t, prev, e))
-                    prev = e
-            if merge_layers is not None:
-                for t in range(C):
-                    for l in range(R):
-                        merge_layers[l].step(xs[l], t, outs[l][t], side)
-                        prev = ev()
-                for l in range(R):
-                    merge_layers[l].merge(side)
-                    e = ev()
-                    recs.append(("merge", C, prev, e))
-                    prev = e
-    stream.wait_stream(side)
+    ios = [[io(t, l) for l in range(R)] for t in range(C)]
+    plan = []                                   # (kind, t, callable)
+    for t in range(C):
+        for l in range(R):
+            h = layers[l].handle.h
+            plan.append(("merge_token" if t == C - 1 else "append", t,
+                         (lib.dl_decode_step, (h,) + ios[t][l] + (st,))))
+    if merge_layers is not None:
+        for t in range(C):
+            for l in range(R):
+                plan.append((None, t, (lib.dl_decode_step,
+                                       (merge_layers[l].handle.h,) + ios[t][l] + (st,))))
+        for l in range(R):
+            plan.append(("merge", C, (lib.dl_merge, (merge_layers[l].handle.h, st))))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(plan) + 1)]
     out = {}
-    g.replay()                       # warm-up
-    torch.cuda.synchronize(dev)
-    for _ in range(reps):
-        g.replay()
+    for rep in range(reps + 1):
+        prime()
+        evs[0].record(stream)
+        for i, (kind, t, (fn, args)) in enumerate(plan):
+            rc = fn(*args)
+            if rc != B.DL_OK:
+                raise RuntimeError(f"launch failed: {B.dl_strerror(rc)}: {B.dl_last_error()}")
+            evs[i + 1].record(stream)
         torch.cuda.synchronize(dev)
-        for kind, t, a, b in recs:
-            out.setdefault((kind, t), []).append(a.elapsed_time(b))
-    del g
+        if rep == 0:
+            continue                             # warm-up
+        for i, (kind, t, _) in enumerate(plan):
+            if kind is not None:
+                out.setdefault((kind, t), []).append(evs[i].elapsed_time(evs[i + 1]))
     return out
 
 
@@ -399,7 +401,7 @@ def run_native(args, rank, world, local_rank):
     # --- per-kernel durations, CUDA events inside a replayed graph
     merge_layers = _layers(w, R, rank, dev, B.DL_MERGE_OFF)
     kd = kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps=max(3, min(args.steps, 10)),
-                          merge_layers=merge_layers)
+                          prime=lambda: cycle.launch(stream), merge_layers=merge_layers)
     app = {t: statistics.mean(kd[("append", t)]) for t in range(C - 1) if ("append", t) in kd}
     fold_us = statistics.mean(kd[("merge_token", C - 1)]) * 1e3 if ("merge_token", C - 1) in kd else None
     merge_us = statistics.mean(kd[("merge", C)]) * 1e3
