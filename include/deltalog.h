@@ -97,13 +97,19 @@ typedef struct dl_handle dl_handle;   /* opaque; host memory only */
  *                                  in_dtype copies of v (RWKV6)
  *   Lambda float [NH, C, m]        cumulative log-decay since the last merge,
  *                                  m = 1 (GDN) or d_k (KDA, RWKV6)
+ *   status uint32 (256 bytes)      device-side error bits: bit 0 is set when a
+ *                                  kernel gave up waiting for its bulk copies
+ *                                  (after 2 s) and returned without computing;
+ *                                  zero it with the workspace, read it after a
+ *                                  synchronisation if in doubt
  * The log is the paper's "bounded update log" (gist.science technical
  * summary, "Meccanismo Core: Base + Log"). */
 size_t dl_log_bytes(const dl_config *cfg);
 
-/* Byte offsets of the K, U and Lambda regions inside the log workspace. */
+/* Byte offsets of the K, U, Lambda and status regions of the workspace
+ * (any output pointer may be NULL). */
 dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U,
-                        size_t *off_Lam);
+                        size_t *off_Lam, size_t *off_status);
 
 /* Create a decode handle over a caller-owned base state (device, fp32
  * [NH, d_k, d_v], 16-byte aligned, holds S at the last merge) and log

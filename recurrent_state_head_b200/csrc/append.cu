@@ -8,12 +8,13 @@ namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
-    constexpr int NT = 4 * TV;
+    constexpr int NT = (TV == 32) ? 128 : 256;
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD>;
     const int ie = p.in_bf16 ? 2 : 4;
-    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
-    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
+    const size_t smem = smem_layout<OP, DK, DV, TV, NT>(p.L, ie, true, FOLD, FOLD).bytes;
+    cudaError_t e =
+        allow_smem(smem_ok, kern, smem_layout<OP, DK, DV, TV, NT>(MAXC - 1, 4, true, FOLD, FOLD).bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)p.NH * (DV / TV);
     kern<<<grid, NT, smem, s>>>(p);

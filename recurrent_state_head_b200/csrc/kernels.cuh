@@ -41,6 +41,7 @@ struct AppendParams {
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
+    unsigned *status;         // error word in the log workspace
 };
 
 struct MergeParams {
@@ -51,6 +52,7 @@ struct MergeParams {
     const float *logLam;
     int NH, C, L;
     int in_bf16;
+    unsigned *status;         // error word in the log workspace
 };
 
 struct EagerParams {
@@ -188,97 +190,181 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
-// ===================================================== operand staging ==
+// ===================================================== TMA bulk staging ==
 //
-// The append, merge-token and merge kernels hold their base tile in
-// registers (16-byte loads issued first, so they are in flight while
-// everything else happens) and stage the small operands -- the token's rows,
-// its decay, beta or bonus, and the L logged entries -- in dynamic shared
-// memory with cp.async issued by warp 0 alone, waited for with
-// cp.async.wait_all (a hardware wait) and published with __syncthreads.
+// The append, merge-token and merge kernels land everything they read --
+// the base tile and the small operands -- in shared memory with TMA bulk
+// copies (cp.async.bulk, one instruction per contiguous chunk: a whole head
+// is one copy), completing on one mbarrier per CTA.  Landing the stream in
+// shared memory rather than registers lets a few resident CTAs keep
+// ~150-200 KB of reads in flight per SM, which a pure read stream needs to
+// run at HBM rate.  Thread 0 waits on the mbarrier with a time bound; on
+// timeout the CTA records an error in the status word and returns.
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar` for at most `limit_ns`; false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity,
+                                                  unsigned long long limit_ns) {
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// Bulk copy global -> shared (both 16-byte aligned, size a multiple of 16),
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr unsigned kStatusTimeout = 1u;
 
 __host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
-// Byte offsets of the staged operands (all 16-byte aligned).
-struct OpLayout {
-    int kin, qin, vin, g, beta, bonus, K, lam, U, A, bytes;
+// Shared-memory layout of one CTA (byte offsets, 16-byte aligned).  `tx` is
+// the byte count the bulk copies deliver (the mbarrier's transaction count).
+struct SmemLayout {
+    int tile, kin, qin, vin, g, bonus, K, lam, U, A, red, bytes, tx;
 };
 
-// token: stage the token's k, q (r), v tile, g, beta / bonus.  A: room for
-// the [DK][up4(L) + 4] fp32 table of per-row replay factors (merge,
-// merge-token).
-template <int OP, int DK, int TV>
-__host__ __device__ inline OpLayout op_layout(int L, int ie, bool token, bool table) {
-    const int M = (OP == OP_GDN) ? 1 : DK;
+// token: the token's k, q (r), v tile, g and (RWKV6) bonus.  table: the
+// [DK][up4(L) + 4] replay-factor table.  red: a separate region for the
+// row partials (when the tile must survive the reduction).
+template <int OP, int DK, int DV, int TV, int NT>
+__host__ __device__ inline SmemLayout smem_layout(int L, int ie, bool token, bool table, bool red) {
+    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
-    OpLayout s{};
-    int o = 0;
-    s.kin = o; o += token ? up16(DK * ie) : 0;
-    s.qin = o; o += token ? up16(DK * ie) : 0;
-    s.vin = o; o += token ? up16(TV * ie) : 0;
-    s.g = o; o += token ? up16(M * 4) : 0;
-    s.beta = o; o += token ? 16 : 0;
-    s.bonus = o; o += (token && OP == OP_RWKV6) ? DK * 4 : 0;
-    s.K = o; o += up16(L * DK * ie);
-    s.lam = o; o += up16(L * M * 4);
-    s.U = o; o += up16(L * TV * ue);
-    s.A = o; o += table ? DK * (up4(L) + 4) * 4 : 0;
+    SmemLayout s{};
+    int o = 0, tx = 0;
+    s.tile = o; o += DK * TV * 4; tx += DK * TV * 4;
+    s.kin = o; if (token) { o += DK * ie; tx += DK * ie; }
+    s.qin = o; if (token) { o += DK * ie; tx += DK * ie; }
+    s.vin = o; if (token) { o += TV * ie; tx += TV * ie; }
+    s.g = o; if (token && M > 1) { o += M * 4; tx += M * 4; }
+    s.bonus = o; if (token && OP == OP_RWKV6) { o += DK * 4; tx += DK * 4; }
+    s.K = o; o += L * DK * ie; tx += L * DK * ie;
+    s.lam = o; if (M > 1) { o += L * M * 4; tx += L * M * 4; }
+    s.U = o; o += L * TV * ue; tx += L * TV * ue;
+    o = up16(o);
+    s.A = o; if (table) o += DK * (up4(L) + 4) * 4;
+    s.red = o; if (red) o += NA * (NT / 32) * TV * 4;
     s.bytes = o;
+    s.tx = tx;
     return s;
 }
 
-// warp-level copy of `bytes` (a multiple of 16; 16-byte aligned addresses)
-__device__ __forceinline__ void warp_copy(unsigned char *dst, const void *src, int bytes, int lane) {
-    const char *g = static_cast<const char *>(src);
-    for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, g + o);
-}
-
-// Sources of one head's staged operands.
+// Sources of one unit's operands.
 struct OpSources {
-    const void *k, *q, *v;          // token rows (NULL: not staged)
-    const float *g, *beta, *bonus;
+    const float *base;
+    const void *k, *q, *v;          // token rows (unused without `token`)
+    const float *g, *bonus;
     const void *logK, *logU;
     const float *logLam;
 };
 
-// Stage one unit's operands (warp 0 only), then wait for them.
+// Issue the bulk copies of one unit (warp 0; lane 0 has armed the barrier).
 template <int OP, int DK, int DV, int TV>
-__device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay, const OpSources &src,
-                                          int head, int vt, int L, int C, int H, int ie, bool token) {
+__device__ __forceinline__ void issue_bulk(unsigned char *sm, const SmemLayout &lay, const OpSources &src,
+                                           int head, int vt, int L, int C, int H, int ie, bool token,
+                                           uint64_t *bar) {
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
     const int lane = threadIdx.x & 31;
-    if (token) {
-        warp_copy(sm + lay.kin, static_cast<const char *>(src.k) + (size_t)head * DK * ie, DK * ie, lane);
-        warp_copy(sm + lay.qin, static_cast<const char *>(src.q) + (size_t)head * DK * ie, DK * ie, lane);
-        warp_copy(sm + lay.vin, static_cast<const char *>(src.v) + ((size_t)head * DV + vt * TV) * ie,
-                  TV * ie, lane);
-        if (OP == OP_GDN) {
-            if (lane == 0) cp_async4(sm + lay.g, src.g + head);
-        } else {
-            warp_copy(sm + lay.g, src.g + (size_t)head * DK, DK * 4, lane);
-        }
-        if (OP == OP_RWKV6)
-            warp_copy(sm + lay.bonus, src.bonus + (size_t)(head % H) * DK, DK * 4, lane);
-        else if (lane == 1)
-            cp_async4(sm + lay.beta, src.beta + head);
-    }
-    warp_copy(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie, L * DK * ie,
-              lane);
-    const float *lamh = src.logLam + (size_t)head * C * M;
-    if (OP == OP_GDN) {
-        for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
+    const float *bt = src.base + (size_t)head * DK * DV + vt * TV;
+    if (TV == DV) {
+        if (lane == 0) bulk_load(sm + lay.tile, bt, DK * DV * 4, bar);
     } else {
-        warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
+        for (int r = lane; r < DK; r += 32)
+            bulk_load(sm + lay.tile + r * TV * 4, bt + (size_t)r * DV, TV * 4, bar);
     }
-    const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
-    const int cpr = TV * ue / 16;
-    for (int idx = lane; idx < L * cpr; idx += 32) {
-        const int j = idx / cpr, c = idx - j * cpr;
-        cp_async16(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16);
+    if (token) {
+        if (lane == 1)
+            bulk_load(sm + lay.kin, static_cast<const char *>(src.k) + (size_t)head * DK * ie, DK * ie, bar);
+        if (lane == 2)
+            bulk_load(sm + lay.qin, static_cast<const char *>(src.q) + (size_t)head * DK * ie, DK * ie, bar);
+        if (lane == 3)
+            bulk_load(sm + lay.vin, static_cast<const char *>(src.v) + ((size_t)head * DV + vt * TV) * ie,
+                      TV * ie, bar);
+        if (M > 1 && lane == 4) bulk_load(sm + lay.g, src.g + (size_t)head * DK, DK * 4, bar);
+        if (OP == OP_RWKV6 && lane == 5)
+            bulk_load(sm + lay.bonus, src.bonus + (size_t)(head % H) * DK, DK * 4, bar);
     }
-    cp_async_wait_all();
+    if (L > 0) {
+        if (lane == 6)
+            bulk_load(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie,
+                      L * DK * ie, bar);
+        if (M > 1 && lane == 7)
+            bulk_load(sm + lay.lam, src.logLam + (size_t)head * C * M, L * M * 4, bar);
+        const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
+        if (TV == DV) {
+            if (lane == 8) bulk_load(sm + lay.U, lU, L * DV * ue, bar);
+        } else {
+            for (int j = lane; j < L; j += 32)
+                bulk_load(sm + lay.U + j * TV * ue, lU + (size_t)j * DV * ue, TV * ue, bar);
+        }
+    }
+}
+
+// Arm the CTA's barrier, issue the copies, wait (thread 0, bounded).  All
+// threads return the same verdict; on timeout the status word is set.
+template <int OP, int DK, int DV, int TV>
+__device__ __forceinline__ bool stage_unit(unsigned char *sm, const SmemLayout &lay, const OpSources &src,
+                                           int head, int vt, int L, int C, int H, int ie, bool token,
+                                           uint64_t *bar, int *s_ok, unsigned *status) {
+    if (threadIdx.x == 0) mbar_init(bar, 1);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, (unsigned)lay.tx);
+        __syncwarp();
+        issue_bulk<OP, DK, DV, TV>(sm, lay, src, head, vt, L, C, H, ie, token, bar);
+    }
+    if (threadIdx.x == 0) {
+        bool ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
+        if (!ok) {
+            atomicOr(status, kStatusTimeout);
+            mbar_wait_bounded(bar, 0, kWaitLimitNs);   // give copies in flight a last chance to land
+        }
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
 }
 
 // Four consecutive elements of a raw vector in shared memory as fp32.
@@ -309,7 +395,7 @@ __device__ __forceinline__ void replay_table(float *A, float *gam, const float *
     }
 }
 
-// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3] (+ kr * w4)
+// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3]
 template <int TV>
 __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow, const unsigned char *sU,
                                            int c4, int L, int ubf) {
@@ -338,15 +424,14 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
 // (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
 // Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
 // (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
-// x = Sbar^T w over the register tile (the one base read), value-side replay,
+// x = Sbar^T w over the staged tile (the one base read), value-side replay,
 // delta correction, output.
 // FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
 //   slot L; the base is not written.
 // FOLD = true (merge-token, the step that completes the log: "Fase di
 //   Merge"): the logical state after this token -- base decayed to Lambda_t,
 //   all L logged factors and this token's k u^T -- is written over the base
-//   tile (the register tile is read once and written once); the log is left
-//   for the caller to reset (L = 0).
+//   tile (read once, written once); the caller resets the log (L = 0).
 template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
@@ -355,7 +440,12 @@ append_kernel(const AppendParams p) {
     constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
-    extern __shared__ __align__(16) unsigned char dsm[];
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ uint64_t s_bar;
+    __shared__ int s_ok;
+    __shared__ float s_gsc;              // GDN: the token's scalar log-decay
+    __shared__ float s_beta;
+    __shared__ float s_lamg[MAXC];       // GDN: logged scalar snapshots
     __shared__ float s_lt[DK];           // Lambda_t
     __shared__ float s_lr[DK];           // decay point of read-out and replay
     __shared__ float s_k[DK];
@@ -365,7 +455,6 @@ append_kernel(const AppendParams p) {
     __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
-    __shared__ __align__(16) float s_red[NA * T::NW * TV];
     __shared__ float s_x[NA * TV];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
@@ -376,24 +465,25 @@ append_kernel(const AppendParams p) {
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
+    const SmemLayout lay = smem_layout<OP, DK, DV, TV, NT>(L, ie, true, FOLD, FOLD);
 
-    // 1. the base stream: RPT rows x 16 bytes per thread
-    float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
-    float4 s[T::RPT];
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r)
-        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
-                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
-
-    // 2. small operands, staged by warp 0 while the base loads are in flight
-    if (tid < 32) {
-        const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
-        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true);
+    // 1. scalars the bulk copies do not carry (plain loads, overlapping the copies)
+    if (OP == OP_GDN) {
+        if (tid == 32) s_gsc = p.g[head];
+        for (int j = tid - 64; j >= 0 && j < L; j += NT) s_lamg[j] = p.logLam[(size_t)head * C + j];
     }
-    __syncthreads();
-    const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
-    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
+    if (OP != OP_RWKV6 && tid == 33) s_beta = p.beta[head];
+
+    // 2. the base tile and the small operands, bulk-copied into shared memory
+    {
+        const OpSources src{p.base, p.k, p.q, p.v, p.g, p.bonus, p.logK, p.logU, p.logLam};
+        if (!stage_unit<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true, &s_bar, &s_ok,
+                                        p.status))
+            return;
+    }
+    const float *tile = reinterpret_cast<const float *>(dsm + lay.tile);
+    const float *slam = (OP == OP_GDN) ? s_lamg : reinterpret_cast<const float *>(dsm + lay.lam);
+    const float *sg = (OP == OP_GDN) ? &s_gsc : reinterpret_cast<const float *>(dsm + lay.g);
 
     // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
     if (tid < DK) {
@@ -460,7 +550,7 @@ append_kernel(const AppendParams p) {
                                        dsm + lay.K, slam, L, p.in_bf16);
     __syncthreads();
 
-    // 4. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    // 4. base read-out from the staged tile: x_a[c] = sum_i w_a[i] * Sbar[i][c]
     {
         float4 acc[NA];
 #pragma unroll
@@ -468,16 +558,19 @@ append_kernel(const AppendParams p) {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
+            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
                 const float w = s_w[a][row];
-                acc[a].x = fmaf(w, s[r].x, acc[a].x);
-                acc[a].y = fmaf(w, s[r].y, acc[a].y);
-                acc[a].z = fmaf(w, s[r].z, acc[a].z);
-                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+                acc[a].x = fmaf(w, sv.x, acc[a].x);
+                acc[a].y = fmaf(w, sv.y, acc[a].y);
+                acc[a].z = fmaf(w, sv.z, acc[a].z);
+                acc[a].w = fmaf(w, sv.w, acc[a].w);
             }
         }
-        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
+        float *red = reinterpret_cast<float *>(dsm + (FOLD ? lay.red : lay.tile));
+        if (!FOLD) __syncthreads();      // the partials overwrite the consumed tile
+        reduce_rows<NA, TV, NT>(acc, red, s_x);
     }
 
     // 5. value side: log replay, delta correction, output, append of u
@@ -504,8 +597,7 @@ append_kernel(const AppendParams p) {
                 rk = fmaf(s_coef[0][j], uj, rk);
                 rq = fmaf(s_coef[1][j], uj, rq);
             }
-            const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
-            const float u = beta * (vv - s_x[c] - rk);
+            const float u = s_beta * (vv - s_x[c] - rk);
             const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
@@ -522,10 +614,12 @@ append_kernel(const AppendParams p) {
         const int AP = up4(L) + 4;
         const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
         const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
-#pragma unroll
+        float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+#pragma unroll 4
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
-            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
+            float4 o = fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
             const float kr = s_k[row];
             o.x = fmaf(kr, u4.x, o.x);
             o.y = fmaf(kr, u4.y, o.y);
@@ -541,17 +635,19 @@ append_kernel(const AppendParams p) {
 // dst[i][c] = exp(Lambda_L[i]) base[i][c] + sum_{j<L} exp(Lambda_L[i] - Lambda_j[i]) k_j[i] u_j[c]
 // (Lambda_L = the last entry's snapshot; L = 0 copies the base).  In place
 // (dst == base) it is the merge; into another buffer it is materialise.
-// One CTA per unit; the register tile is loaded first, the log staged by
-// warp 0, the replay-factor table built once per CTA.
+// One CTA per unit: the tile and the log land in shared memory by bulk
+// copy, the replay-factor table is built once per CTA.
 template <int OP, int DK, int DV, int TV, int NT>
 __global__ void __launch_bounds__(NT)
 merge_kernel(const MergeParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
 
-    extern __shared__ __align__(16) unsigned char dsm[];
+    extern __shared__ __align__(128) unsigned char dsm[];
+    __shared__ uint64_t s_bar;
+    __shared__ int s_ok;
+    __shared__ float s_lamg[MAXC];
     __shared__ float s_gam[DK];
-    __shared__ float s_lL[M];
 
     const int unit = blockIdx.x;
     const int head = unit / T::NVT, vt = unit - head * T::NVT;
@@ -560,33 +656,43 @@ merge_kernel(const MergeParams p) {
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, false, true);
+    const SmemLayout lay = smem_layout<OP, DK, DV, TV, NT>(L, ie, false, true, false);
 
-    const float *bh = p.base + (size_t)head * DK * DV + vt * TV + c4;
-    float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
-    float4 s[T::RPT];
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
-
-    if (tid < 32) {
-        const OpSources src{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
-        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false);
+    if (OP == OP_GDN)
+        for (int j = tid - 32; j >= 0 && j < L; j += NT) s_lamg[j] = p.logLam[(size_t)head * C + j];
+    {
+        const OpSources src{p.base, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
+        if (!stage_unit<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false, &s_bar, &s_ok,
+                                        p.status))
+            return;
+    }
+    const float *slam = (OP == OP_GDN) ? s_lamg : reinterpret_cast<const float *>(dsm + lay.lam);
+    float *A = reinterpret_cast<float *>(dsm + lay.A);
+    // Lambda_L per key row: the last snapshot (zero for an empty log)
+    const float *lamL = (L > 0) ? slam + (L - 1) * M : nullptr;
+    {
+        const int AP = up4(L) + 4;
+        for (int idx = tid; idx < DK * (L + 1); idx += NT) {
+            const int i = idx % DK, j = idx / DK;
+            const int x = (OP == OP_GDN) ? 0 : i;
+            const float lL = lamL ? lamL[x] : 0.f;
+            if (j == L)
+                s_gam[i] = expf(lL);
+            else
+                A[i * AP + j] = expf(lL - slam[j * M + x]) * ld_raw(dsm + lay.K, j * DK + i, p.in_bf16);
+        }
     }
     __syncthreads();
-    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
-    for (int x = tid; x < M; x += NT) s_lL[x] = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-    __syncthreads();
-    replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lL, dsm + lay.K, slam, L,
-                             p.in_bf16);
-    __syncthreads();
 
-    const float *A = reinterpret_cast<const float *>(dsm + lay.A);
+    const float *tile = reinterpret_cast<const float *>(dsm + lay.tile);
+    float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-#pragma unroll
+#pragma unroll 4
     for (int r = 0; r < T::RPT; ++r) {
         const int row = rg + r * T::RG;
-        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
+        st_state(dh + (size_t)row * DV, fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
     }
 }
 

@@ -87,9 +87,14 @@ class DecodeLayer:
     def merge(self, stream=None):
         self.handle.merge(stream)
 
+    def device_status(self) -> int:
+        """The workspace's device-side error bits (0 when all is well)."""
+        _, _, _, oS = B.dl_log_layout(self.cfg)
+        return int(self.log[oS:oS + 4].view(torch.int32).item())
+
     def log_views(self):
         """(K, U, Lambda) views of the log workspace for inspection."""
-        oK, oU, oL = B.dl_log_layout(self.cfg)
+        oK, oU, oL, _ = B.dl_log_layout(self.cfg)
         NH, C, dk, dv, m = self.w.heads, self.cfg.C, self.w.dk, self.w.dv, self.w.m
         in_t = TORCH_DTYPE[self.w.in_dtype]
         u_t = in_t if self.w.op == RWKV6 else torch.float32
