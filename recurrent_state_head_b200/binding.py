@@ -128,7 +128,7 @@ def dl_log_bytes(cfg: dl_config) -> int:
 
 
 def dl_log_layout(cfg: dl_config):
-    """(offset of K, of U, of Lambda, of the status word) in the workspace."""
+    """(offset of K, of U, of Lambda, of the prep area) in the workspace."""
     a, b, c, d = (ctypes.c_size_t() for _ in range(4))
     _check(lib().dl_log_layout(ctypes.byref(cfg), ctypes.byref(a), ctypes.byref(b),
                                ctypes.byref(c), ctypes.byref(d)))

@@ -62,7 +62,7 @@ dl_status check_config(const dl_config *c, bool need_log) {
 }
 
 struct Layout {
-    size_t K, U, Lam, status, total;
+    size_t K, U, Lam, prep, total;
 };
 
 Layout log_layout(const dl_config *c) {
@@ -73,8 +73,8 @@ Layout log_layout(const dl_config *c) {
     l.K = 0;
     l.U = up256(l.K + nh * C * c->dk * esize(c->in_dtype));
     l.Lam = up256(l.U + nh * C * c->dv * ue);
-    l.status = up256(l.Lam + nh * C * m * 4);
-    l.total = l.status + 256;
+    l.prep = up256(l.Lam + nh * C * m * 4);
+    l.total = up256(l.prep + nh * (size_t)dl::prep_stride(c->op, c->dk) * 4);
     return l;
 }
 
@@ -135,7 +135,8 @@ dl::AppendParams append_params(const dl_handle *h, const dl_step_io &io, int L) 
     p.scale = h->cfg.scale;
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
     p.out_bf16 = h->cfg.out_dtype == DL_BF16;
-    p.status = reinterpret_cast<unsigned *>(h->log + h->lay.status);
+    p.prep = reinterpret_cast<float *>(h->log + h->lay.prep);
+    p.ps = dl::prep_stride(h->cfg.op, h->cfg.dk);
     return p;
 }
 
@@ -150,7 +151,6 @@ dl::MergeParams merge_params(const dl_handle *h, float *dst, int L) {
     p.C = h->cfg.C;
     p.L = L;
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
-    p.status = reinterpret_cast<unsigned *>(h->log + h->lay.status);
     return p;
 }
 
@@ -176,14 +176,14 @@ size_t dl_log_bytes(const dl_config *cfg) {
 }
 
 dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U, size_t *off_Lam,
-                        size_t *off_status) {
+                        size_t *off_prep) {
     dl_status s = check_config(cfg, true);
     if (s != DL_OK) return s;
     const Layout l = log_layout(cfg);
     if (off_K) *off_K = l.K;
     if (off_U) *off_U = l.U;
     if (off_Lam) *off_Lam = l.Lam;
-    if (off_status) *off_status = l.status;
+    if (off_prep) *off_prep = l.prep;
     return ok();
 }
 

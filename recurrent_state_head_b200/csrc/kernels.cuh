@@ -7,14 +7,24 @@
 // with shared key-side metadata and the ReplayPrep / AppendDecode stages
 // ("Implementazione del Kernel"), operators GDN / KDA / RWKV6.
 //
-// Decomposition.  A work unit is one head, or one value tile of a head when
-// there are too few heads to fill the GPU (the paper's value-tile split): TV
-// value columns of all d_k rows, so the key-side contractions S^T x reduce
-// inside the CTA.  NT = 4 TV threads: TV/4 threads per row, each owning a
-// 16-byte column group, 16 row groups, RPT = d_k / 16 rows per thread held in
-// registers.  The eager kernel always uses 32-column tiles.  Nothing here is a dense contraction worth a tensor
-// core: per state element the append does 2 FMAs and the merge at most
-// C = 16, against 4 to 8 bytes of HBM traffic.
+// Staged execution, as in the paper: a decode token is two kernels.
+//   ReplayPrep   one CTA per head: the key-side quantities of the token --
+//                decay point, read-out weights, the L replay coefficients and
+//                the self term -- computed once per head into the prep area
+//                of the log workspace; it also appends k_t and Lambda_t to
+//                the log.
+//   AppendDecode one CTA per (head, value tile) (the paper's value-tile
+//                parallelism): streams its tile of the base, reduces S^T w,
+//                replays the log on the value side and writes the output and
+//                u_t.  It is launched as a programmatic dependent of
+//                ReplayPrep: its base loads are issued before it waits for
+//                ReplayPrep's results, so the prep work hides under the base
+//                stream.
+// Tile geometry: TV value columns of all d_k rows, TV/4 threads per row each
+// owning a 16-byte column group, RPT rows per thread held in registers.
+// Nothing here is a dense contraction worth a tensor core: per state element
+// the append does 2 FMAs and the merge at most C = 16, against 4 to 8 bytes
+// of HBM traffic.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -38,10 +48,11 @@ struct AppendParams {
     const float *g;           // [NH, m]
     const float *bonus;       // [H, DK]
     void *out;                // [NH, DV] out dtype
+    float *prep;              // [NH, ps] ReplayPrep results (log workspace)
+    int ps;                   // prep stride per head (floats)
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
-    unsigned *status;         // error word in the log workspace
 };
 
 struct MergeParams {
@@ -52,7 +63,6 @@ struct MergeParams {
     const float *logLam;
     int NH, C, L;
     int in_bf16;
-    unsigned *status;         // error word in the log workspace
 };
 
 struct EagerParams {
@@ -190,181 +200,197 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
-// ===================================================== TMA bulk staging ==
+// ========================================================= prep layout ==
 //
-// The append, merge-token and merge kernels land everything they read --
-// the base tile and the small operands -- in shared memory with TMA bulk
-// copies (cp.async.bulk, one instruction per contiguous chunk: a whole head
-// is one copy), completing on one mbarrier per CTA.  Landing the stream in
-// shared memory rather than registers lets a few resident CTAs keep
-// ~150-200 KB of reads in flight per SM, which a pure read stream needs to
-// run at HBM rate.  Thread 0 waits on the mbarrier with a time bound; on
-// timeout the CTA records an error in the status word and returns.
-
-__device__ __forceinline__ unsigned smem_u32(const void *p) {
-    return static_cast<unsigned>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
-    unsigned ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for phase `parity` of `bar` for at most `limit_ns`; false on timeout.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity,
-                                                  unsigned long long limit_ns) {
-    const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > limit_ns) return false;
-    return true;
-}
-
-// Bulk copy global -> shared (both 16-byte aligned, size a multiple of 16),
-// completion counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
-constexpr unsigned kStatusTimeout = 1u;
+// Per-head ReplayPrep results, in floats from the head's prep row:
+//   w     [NA][DK]    read-out weights (Gamma_t * k, Gamma_t * q; RWKV6:
+//                     Gamma_{t-1} * r)
+//   coef  [NA][MAXC]  replay coefficients c_j, d_j (RWKV6: d_j) for j < L
+//   self              k.q (RWKV6: r.(bonus * k))
+//   lt    [M]         Lambda_t (used by the merge-token step)
 
 __host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
-// Shared-memory layout of one CTA (byte offsets, 16-byte aligned).  `tx` is
-// the byte count the bulk copies deliver (the mbarrier's transaction count).
-struct SmemLayout {
-    int tile, kin, qin, vin, g, bonus, K, lam, U, A, red, bytes, tx;
+template <int OP, int DK>
+struct PrepLayout {
+    static constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    static constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
+    static constexpr int W = 0;
+    static constexpr int COEF = NA * DK;
+    static constexpr int SELF = COEF + NA * MAXC;
+    static constexpr int LT = SELF + 4;
+    static constexpr int HEAD_BYTES = (SELF + 4) * 4;     // w, coef, self: one copy
+    static constexpr int STRIDE = ((LT + M) + 31) / 32 * 32;
 };
 
-// token: the token's k, q (r), v tile, g and (RWKV6) bonus.  table: the
-// [DK][up4(L) + 4] replay-factor table.  red: a separate region for the
-// row partials (when the tile must survive the reduction).
-template <int OP, int DK, int DV, int TV, int NT>
-__host__ __device__ inline SmemLayout smem_layout(int L, int ie, bool token, bool table, bool red) {
+// Prep stride (floats per head) for a runtime op / d_k.
+inline int prep_stride(int op, int dk) {
+    const int na = op == OP_RWKV6 ? 1 : 2, m = op == OP_GDN ? 1 : dk;
+    return ((na * dk + na * MAXC + 4 + m) + 31) / 32 * 32;
+}
+
+// ========================================================== ReplayPrep ==
+//
+// One CTA of DK threads per head, thread i owning key channel i:
+//   Lambda_t[i] = Lambda_{L-1}[i] + g_t[i]   (0 before the first entry)
+//   w           = exp(Lambda_t) * k, exp(Lambda_t) * q   (RWKV6: exp(Lambda_{t-1}) * r)
+//   c_j, d_j    = sum_i k_i (q_i) k_j[i] exp(lam_i - Lambda_j[i])  for j < L
+//   self        = k . q   (RWKV6: r . (bonus * k))
+// and, unless this token is a merge-token, the key-side append of k_t and
+// Lambda_t to log slot L.  All loads are issued together (one latency round).
+template <int OP, int DK, bool APPEND>
+__global__ void __launch_bounds__(DK)
+replay_prep_kernel(const AppendParams p) {
+    using PL = PrepLayout<OP, DK>;
+    constexpr int M = PL::M, NA = PL::NA;
+    constexpr int NW = DK / 32;
+    constexpr int NV = NA * MAXC + 1;
+    __shared__ float s_part[NW][NV];
+
+    // let the decode grid launch (it first streams the base), then wait for
+    // the previous kernel of the stream
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    const int head = blockIdx.x, i = threadIdx.x;
+    const int lane = i & 31, warp = i >> 5;
+    const int L = p.L, C = p.C;
+    const int x = (OP == OP_GDN) ? 0 : i;
+    const float *lamh = p.logLam + (size_t)head * C * M;
+    const size_t kb = (size_t)head * C * DK + i;
+
+    float kj[MAXC], lj[MAXC];
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        kj[j] = 0.f;
+        lj[j] = 0.f;
+        if (j < L) {
+            kj[j] = ld_in(p.logK, kb + (size_t)j * DK, p.in_bf16);
+            lj[j] = lamh[j * M + x];
+        }
+    }
+    const float lprev = L > 0 ? lamh[(L - 1) * M + x] : 0.f;
+    const float gi = p.g[(size_t)head * M + x];
+    const float kf = ld_in(p.k, (size_t)head * DK + i, p.in_bf16);
+    const float qf = ld_in(p.q, (size_t)head * DK + i, p.in_bf16);
+    const float bon = (OP == OP_RWKV6) ? p.bonus[(size_t)(head % p.H) * DK + i] : 0.f;
+
+    const float lt = lprev + gi;
+    const float lr = (OP == OP_RWKV6) ? lprev : lt;
+    const float gam = expf(lr);
+    float *pr = p.prep + (size_t)head * p.ps;
+    if (OP == OP_RWKV6) {
+        pr[PL::W + i] = gam * qf;
+    } else {
+        pr[PL::W + i] = gam * kf;
+        pr[PL::W + DK + i] = gam * qf;
+    }
+    if (OP != OP_GDN || i == 0) pr[PL::LT + x] = lt;
+    if (APPEND) {
+        copy_in(p.logK, kb + (size_t)L * DK, p.k, (size_t)head * DK + i, p.in_bf16);
+        if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
+    }
+
+    // per-thread terms of the coefficient dot products, reduced over the CTA
+    float part[NV];
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const float e = (OP == OP_GDN) ? kj[j] : expf(lr - lj[j]) * kj[j];
+        if (OP == OP_RWKV6) {
+            part[j] = qf * e;
+        } else {
+            part[j] = kf * e;
+            part[MAXC + j] = qf * e;
+        }
+    }
+    part[NV - 1] = (OP == OP_RWKV6) ? qf * bon * kf : kf * qf;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+        const int j = v % MAXC;
+        if (v == NV - 1 || j < L) {
+            const float s = warp_sum(part[v]);
+            if (lane == 0) s_part[warp][v] = s;
+        }
+    }
+    __syncthreads();
+    for (int v = i; v < NV; v += DK) {
+        const int j = v % MAXC;
+        if (v != NV - 1 && j >= L) continue;
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) s += s_part[w][v];
+        if (OP == OP_GDN && v != NV - 1) s *= expf(lt - lamh[j]);   // scalar decay of entry j
+        pr[PL::COEF + v] = s;                                      // coef[a][j] and self
+    }
+}
+
+// ===================================================== operand staging ==
+//
+// The decode, merge-token and merge kernels hold their base tile in
+// registers (16-byte loads issued first) and stage the small operands in
+// dynamic shared memory with cp.async issued by warp 0 alone, waited for
+// with cp.async.wait_all (a hardware wait) and published with __syncthreads.
+
+// Byte offsets of the staged operands (all 16-byte aligned).
+struct OpLayout {
+    int prep, lt, kin, vin, beta, K, lam, U, A, bytes;
+};
+
+// decode: the head's prep row (w, coef, self), v tile, beta, the tile's L
+// value factors.  fold adds Lambda_t, k and the L logged keys and decay
+// snapshots, and the [DK][up4(L) + 4] replay-factor table.  merge: the log
+// entries and the table only.
+template <int OP, int DK, int TV>
+__host__ __device__ inline OpLayout op_layout(int L, int ie, bool decode, bool fold) {
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
-    constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
-    SmemLayout s{};
-    int o = 0, tx = 0;
-    s.tile = o; o += DK * TV * 4; tx += DK * TV * 4;
-    s.kin = o; if (token) { o += DK * ie; tx += DK * ie; }
-    s.qin = o; if (token) { o += DK * ie; tx += DK * ie; }
-    s.vin = o; if (token) { o += TV * ie; tx += TV * ie; }
-    s.g = o; if (token && M > 1) { o += M * 4; tx += M * 4; }
-    s.bonus = o; if (token && OP == OP_RWKV6) { o += DK * 4; tx += DK * 4; }
-    s.K = o; o += L * DK * ie; tx += L * DK * ie;
-    s.lam = o; if (M > 1) { o += L * M * 4; tx += L * M * 4; }
-    s.U = o; o += L * TV * ue; tx += L * TV * ue;
-    o = up16(o);
-    s.A = o; if (table) o += DK * (up4(L) + 4) * 4;
-    s.red = o; if (red) o += NA * (NT / 32) * TV * 4;
+    const bool logkeys = fold || !decode;
+    OpLayout s{};
+    int o = 0;
+    s.prep = o; o += decode ? PrepLayout<OP, DK>::HEAD_BYTES : 0;
+    s.lt = o; o += fold ? up16(M * 4) : 0;
+    s.kin = o; o += fold ? up16(DK * ie) : 0;
+    s.vin = o; o += decode ? up16(TV * ie) : 0;
+    s.beta = o; o += decode ? 16 : 0;
+    s.K = o; o += logkeys ? up16(L * DK * ie) : 0;
+    s.lam = o; o += logkeys ? up16(L * M * 4) : 0;
+    s.U = o; o += up16(L * TV * ue);
+    s.A = o; o += logkeys ? DK * (up4(L) + 4) * 4 : 0;
     s.bytes = o;
-    s.tx = tx;
     return s;
 }
 
-// Sources of one unit's operands.
-struct OpSources {
-    const float *base;
-    const void *k, *q, *v;          // token rows (unused without `token`)
-    const float *g, *bonus;
-    const void *logK, *logU;
-    const float *logLam;
-};
+// warp-level copy of `bytes` (a multiple of 16; 16-byte aligned addresses)
+__device__ __forceinline__ void warp_copy(unsigned char *dst, const void *src, int bytes, int lane) {
+    const char *g = static_cast<const char *>(src);
+    for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, g + o);
+}
 
-// Issue the bulk copies of one unit (warp 0; lane 0 has armed the barrier).
+// Stage the L logged entries of one head / value tile (warp 0).
 template <int OP, int DK, int DV, int TV>
-__device__ __forceinline__ void issue_bulk(unsigned char *sm, const SmemLayout &lay, const OpSources &src,
-                                           int head, int vt, int L, int C, int H, int ie, bool token,
-                                           uint64_t *bar) {
+__device__ __forceinline__ void stage_log(unsigned char *sm, const OpLayout &lay, const void *logK,
+                                          const void *logU, const float *logLam, int head, int vt, int L,
+                                          int C, int ie, bool keys) {
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
     const int lane = threadIdx.x & 31;
-    const float *bt = src.base + (size_t)head * DK * DV + vt * TV;
-    if (TV == DV) {
-        if (lane == 0) bulk_load(sm + lay.tile, bt, DK * DV * 4, bar);
-    } else {
-        for (int r = lane; r < DK; r += 32)
-            bulk_load(sm + lay.tile + r * TV * 4, bt + (size_t)r * DV, TV * 4, bar);
-    }
-    if (token) {
-        if (lane == 1)
-            bulk_load(sm + lay.kin, static_cast<const char *>(src.k) + (size_t)head * DK * ie, DK * ie, bar);
-        if (lane == 2)
-            bulk_load(sm + lay.qin, static_cast<const char *>(src.q) + (size_t)head * DK * ie, DK * ie, bar);
-        if (lane == 3)
-            bulk_load(sm + lay.vin, static_cast<const char *>(src.v) + ((size_t)head * DV + vt * TV) * ie,
-                      TV * ie, bar);
-        if (M > 1 && lane == 4) bulk_load(sm + lay.g, src.g + (size_t)head * DK, DK * 4, bar);
-        if (OP == OP_RWKV6 && lane == 5)
-            bulk_load(sm + lay.bonus, src.bonus + (size_t)(head % H) * DK, DK * 4, bar);
-    }
-    if (L > 0) {
-        if (lane == 6)
-            bulk_load(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie,
-                      L * DK * ie, bar);
-        if (M > 1 && lane == 7)
-            bulk_load(sm + lay.lam, src.logLam + (size_t)head * C * M, L * M * 4, bar);
-        const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
-        if (TV == DV) {
-            if (lane == 8) bulk_load(sm + lay.U, lU, L * DV * ue, bar);
+    if (keys) {
+        warp_copy(sm + lay.K, static_cast<const char *>(logK) + (size_t)head * C * DK * ie, L * DK * ie,
+                  lane);
+        const float *lamh = logLam + (size_t)head * C * M;
+        if (OP == OP_GDN) {
+            for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
         } else {
-            for (int j = lane; j < L; j += 32)
-                bulk_load(sm + lay.U + j * TV * ue, lU + (size_t)j * DV * ue, TV * ue, bar);
+            warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
         }
     }
-}
-
-// Arm the CTA's barrier, issue the copies, wait (thread 0, bounded).  All
-// threads return the same verdict; on timeout the status word is set.
-template <int OP, int DK, int DV, int TV>
-__device__ __forceinline__ bool stage_unit(unsigned char *sm, const SmemLayout &lay, const OpSources &src,
-                                           int head, int vt, int L, int C, int H, int ie, bool token,
-                                           uint64_t *bar, int *s_ok, unsigned *status) {
-    if (threadIdx.x == 0) mbar_init(bar, 1);
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, (unsigned)lay.tx);
-        __syncwarp();
-        issue_bulk<OP, DK, DV, TV>(sm, lay, src, head, vt, L, C, H, ie, token, bar);
+    const char *lU = static_cast<const char *>(logU) + ((size_t)head * C * DV + vt * TV) * ue;
+    const int cpr = TV * ue / 16;
+    for (int idx = lane; idx < L * cpr; idx += 32) {
+        const int j = idx / cpr, c = idx - j * cpr;
+        cp_async16(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16);
     }
-    if (threadIdx.x == 0) {
-        bool ok = mbar_wait_bounded(bar, 0, kWaitLimitNs);
-        if (!ok) {
-            atomicOr(status, kStatusTimeout);
-            mbar_wait_bounded(bar, 0, kWaitLimitNs);   // give copies in flight a last chance to land
-        }
-        *s_ok = ok;
-    }
-    __syncthreads();
-    return *s_ok != 0;
 }
 
 // Four consecutive elements of a raw vector in shared memory as fp32.
@@ -417,18 +443,15 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
     return o;
 }
 
-// ============================================ append + read-out (+ fold) ==
+// ======================================== AppendDecode (+ merge-token) ==
 //
-// One CTA per unit (a head, or a TV-column value tile of a head).
-// ReplayPrep (once per CTA): decay point Lambda_t = Lambda_{L-1} + g_t
-// (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
-// Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
-// (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
-// x = Sbar^T w over the staged tile (the one base read), value-side replay,
-// delta correction, output.
-// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
-//   slot L; the base is not written.
-// FOLD = true (merge-token, the step that completes the log: "Fase di
+// One CTA per (head, value tile), after ReplayPrep: x = Sbar^T w over the
+// register tile (the one base read), value-side replay r = sum_j coef_j u_j,
+// delta correction u = beta (v - x_k - r_k), output o = scale (x_q + r_q +
+// self u) (RWKV6: o = scale (x_r + r_r + self v)).
+// FOLD = false (append, "Fase di Append"): u_t goes to log slot L; the base
+//   is not written.
+// FOLD = true (merge-token, the token that completes the log: "Fase di
 //   Merge"): the logical state after this token -- base decayed to Lambda_t,
 //   all L logged factors and this token's k u^T -- is written over the base
 //   tile (read once, written once); the caller resets the log (L = 0).
@@ -436,26 +459,14 @@ template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
-    constexpr int M = (OP == OP_GDN) ? 1 : DK;
-    constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
+    using PL = PrepLayout<OP, DK>;
+    constexpr int NA = PL::NA;
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
-    extern __shared__ __align__(128) unsigned char dsm[];
-    __shared__ uint64_t s_bar;
-    __shared__ int s_ok;
-    __shared__ float s_gsc;              // GDN: the token's scalar log-decay
-    __shared__ float s_beta;
-    __shared__ float s_lamg[MAXC];       // GDN: logged scalar snapshots
-    __shared__ float s_lt[DK];           // Lambda_t
-    __shared__ float s_lr[DK];           // decay point of read-out and replay
-    __shared__ float s_k[DK];
-    __shared__ float s_q[DK];
-    __shared__ float s_w[NA][DK];        // read-out weights
-    __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
-    __shared__ float s_gam[FOLD ? DK : 1];
-    __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
-    __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ __align__(16) float s_red[NA * T::NW * TV];
     __shared__ float s_x[NA * TV];
+    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
     const int unit = blockIdx.x;
@@ -465,92 +476,46 @@ append_kernel(const AppendParams p) {
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const SmemLayout lay = smem_layout<OP, DK, DV, TV, NT>(L, ie, true, FOLD, FOLD);
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
 
-    // 1. scalars the bulk copies do not carry (plain loads, overlapping the copies)
-    if (OP == OP_GDN) {
-        if (tid == 32) s_gsc = p.g[head];
-        for (int j = tid - 64; j >= 0 && j < L; j += NT) s_lamg[j] = p.logLam[(size_t)head * C + j];
-    }
-    if (OP != OP_RWKV6 && tid == 33) s_beta = p.beta[head];
-
-    // 2. the base tile and the small operands, bulk-copied into shared memory
-    {
-        const OpSources src{p.base, p.k, p.q, p.v, p.g, p.bonus, p.logK, p.logU, p.logLam};
-        if (!stage_unit<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true, &s_bar, &s_ok,
-                                        p.status))
-            return;
-    }
-    const float *tile = reinterpret_cast<const float *>(dsm + lay.tile);
-    const float *slam = (OP == OP_GDN) ? s_lamg : reinterpret_cast<const float *>(dsm + lay.lam);
-    const float *sg = (OP == OP_GDN) ? &s_gsc : reinterpret_cast<const float *>(dsm + lay.g);
-
-    // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
-    if (tid < DK) {
-        const int i = tid;
-        const int x = (OP == OP_GDN) ? 0 : i;
-        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-        const float lt = lprev + sg[x];
-        const float lr = (OP == OP_RWKV6) ? lprev : lt;
-        const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
-        const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
-        const float gam = expf(lr);
-        s_lt[i] = lt;
-        s_lr[i] = lr;
-        s_k[i] = kf;
-        s_q[i] = qf;
-        if (OP == OP_RWKV6) {
-            s_w[0][i] = gam * qf;
-            s_bk[i] = reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf;
-        } else {
-            s_w[0][i] = gam * kf;
-            s_w[NA - 1][i] = gam * qf;
-        }
-        if (!FOLD && vt == 0) {
-            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
-            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
-        }
-    }
-    __syncthreads();
-
-    // replay coefficients: task tau < L is log entry tau, tau == L the self term
-    {
-        const int lane = tid & 31, warp = tid >> 5;
-        for (int tau = warp; tau <= L; tau += T::NW) {
-            float a0 = 0.f, a1 = 0.f;
-            if (tau < L) {
-                const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
+    // 1. the base stream: RPT rows x 16 bytes per thread (independent of
+    //    ReplayPrep, so it starts before waiting for it)
+    float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
 #pragma unroll
-                for (int i = lane; i < DK; i += 32) {
-                    const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
-                    const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
-                    if (OP == OP_RWKV6) {
-                        a0 = fmaf(s_q[i], e, a0);
-                    } else {
-                        a0 = fmaf(s_k[i], e, a0);
-                        a1 = fmaf(s_q[i], e, a1);
-                    }
-                }
-                a0 = warp_sum(a0) * gdec;
-                if (NA == 2) a1 = warp_sum(a1) * gdec;
-                if (lane == 0) {
-                    s_coef[0][tau] = a0;
-                    if (NA == 2) s_coef[NA - 1][tau] = a1;
-                }
+    for (int r = 0; r < T::RPT; ++r)
+        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
+                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+
+    // 2. ReplayPrep's results and the value-side operands
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid < 32) {
+        const int lane = tid;
+        warp_copy(dsm + lay.prep, p.prep + (size_t)head * p.ps, PL::HEAD_BYTES, lane);
+        warp_copy(dsm + lay.vin, static_cast<const char *>(p.v) + ((size_t)head * DV + vt * TV) * ie,
+                  TV * ie, lane);
+        if (OP != OP_RWKV6 && lane == 0) cp_async4(dsm + lay.beta, p.beta + head);
+        if (FOLD) {
+            if (OP == OP_GDN) {
+                if (lane == 1) cp_async4(dsm + lay.lt, p.prep + (size_t)head * p.ps + PL::LT);
             } else {
-#pragma unroll
-                for (int i = lane; i < DK; i += 32)
-                    a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
-                a0 = warp_sum(a0);
-                if (lane == 0) s_self = a0;
+                warp_copy(dsm + lay.lt, p.prep + (size_t)head * p.ps + PL::LT, DK * 4, lane);
             }
+            warp_copy(dsm + lay.kin, static_cast<const char *>(p.k) + (size_t)head * DK * ie, DK * ie, lane);
         }
+        stage_log<OP, DK, DV, TV>(dsm, lay, p.logK, p.logU, p.logLam, head, vt, L, C, ie, FOLD);
+        cp_async_wait_all();
     }
-    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
-                                       dsm + lay.K, slam, L, p.in_bf16);
     __syncthreads();
+    const float *sp = reinterpret_cast<const float *>(dsm + lay.prep);
+    if (FOLD) {
+        replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam,
+                                 reinterpret_cast<const float *>(dsm + lay.lt), dsm + lay.K,
+                                 reinterpret_cast<const float *>(dsm + lay.lam), L, p.in_bf16);
+        __syncthreads();
+    }
 
-    // 4. base read-out from the staged tile: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    // 3. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
     {
         float4 acc[NA];
 #pragma unroll
@@ -558,32 +523,30 @@ append_kernel(const AppendParams p) {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
-            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
-                const float w = s_w[a][row];
-                acc[a].x = fmaf(w, sv.x, acc[a].x);
-                acc[a].y = fmaf(w, sv.y, acc[a].y);
-                acc[a].z = fmaf(w, sv.z, acc[a].z);
-                acc[a].w = fmaf(w, sv.w, acc[a].w);
+                const float w = sp[PL::W + a * DK + row];
+                acc[a].x = fmaf(w, s[r].x, acc[a].x);
+                acc[a].y = fmaf(w, s[r].y, acc[a].y);
+                acc[a].z = fmaf(w, s[r].z, acc[a].z);
+                acc[a].w = fmaf(w, s[r].w, acc[a].w);
             }
         }
-        float *red = reinterpret_cast<float *>(dsm + (FOLD ? lay.red : lay.tile));
-        if (!FOLD) __syncthreads();      // the partials overwrite the consumed tile
-        reduce_rows<NA, TV, NT>(acc, red, s_x);
+        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
     }
 
-    // 5. value side: log replay, delta correction, output, append of u
+    // 4. value side: log replay, delta correction, output, append of u
     if (tid < TV) {
         const int c = tid;
         const int col = vt * TV + c;
         const size_t ub = (size_t)head * C * DV + col;
         const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
+        const float *cf = sp + PL::COEF;
+        const float self = sp[PL::SELF];
         if (OP == OP_RWKV6) {
             float rr = 0.f;
-            for (int j = 0; j < L; ++j)
-                rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
-            const float o = p.scale * (s_x[c] + rr + s_self * vv);
+            for (int j = 0; j < L; ++j) rr = fmaf(cf[j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
+            const float o = p.scale * (s_x[c] + rr + self * vv);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = vv;
@@ -594,11 +557,12 @@ append_kernel(const AppendParams p) {
             float rk = 0.f, rq = 0.f;
             for (int j = 0; j < L; ++j) {
                 const float uj = U[j * TV + c];
-                rk = fmaf(s_coef[0][j], uj, rk);
-                rq = fmaf(s_coef[1][j], uj, rq);
+                rk = fmaf(cf[j], uj, rk);
+                rq = fmaf(cf[MAXC + j], uj, rq);
             }
-            const float u = s_beta * (vv - s_x[c] - rk);
-            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+            const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
+            const float u = beta * (vv - s_x[c] - rk);
+            const float o = p.scale * (s_x[TV + c] + rq + self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = u;
@@ -607,20 +571,18 @@ append_kernel(const AppendParams p) {
         }
     }
 
-    // 6. merge-token: write the logical state after this token over the base
+    // 5. merge-token: write the logical state after this token over the base
     if (FOLD) {
         __syncthreads();
         const float *A = reinterpret_cast<const float *>(dsm + lay.A);
         const int AP = up4(L) + 4;
         const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
         const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
-        float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
-#pragma unroll 4
+#pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
-            const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
-            float4 o = fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-            const float kr = s_k[row];
+            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+            const float kr = ld_raw(dsm + lay.kin, row, p.in_bf16);
             o.x = fmaf(kr, u4.x, o.x);
             o.y = fmaf(kr, u4.y, o.y);
             o.z = fmaf(kr, u4.z, o.z);
@@ -635,19 +597,17 @@ append_kernel(const AppendParams p) {
 // dst[i][c] = exp(Lambda_L[i]) base[i][c] + sum_{j<L} exp(Lambda_L[i] - Lambda_j[i]) k_j[i] u_j[c]
 // (Lambda_L = the last entry's snapshot; L = 0 copies the base).  In place
 // (dst == base) it is the merge; into another buffer it is materialise.
-// One CTA per unit: the tile and the log land in shared memory by bulk
-// copy, the replay-factor table is built once per CTA.
+// One CTA per unit; the register tile is loaded first, the log staged by
+// warp 0, the replay-factor table built once per CTA.
 template <int OP, int DK, int DV, int TV, int NT>
 __global__ void __launch_bounds__(NT)
 merge_kernel(const MergeParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
 
-    extern __shared__ __align__(128) unsigned char dsm[];
-    __shared__ uint64_t s_bar;
-    __shared__ int s_ok;
-    __shared__ float s_lamg[MAXC];
+    extern __shared__ __align__(16) unsigned char dsm[];
     __shared__ float s_gam[DK];
+    __shared__ float s_lL[M];
 
     const int unit = blockIdx.x;
     const int head = unit / T::NVT, vt = unit - head * T::NVT;
@@ -656,43 +616,33 @@ merge_kernel(const MergeParams p) {
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const SmemLayout lay = smem_layout<OP, DK, DV, TV, NT>(L, ie, false, true, false);
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, false, false);
 
-    if (OP == OP_GDN)
-        for (int j = tid - 32; j >= 0 && j < L; j += NT) s_lamg[j] = p.logLam[(size_t)head * C + j];
-    {
-        const OpSources src{p.base, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
-        if (!stage_unit<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false, &s_bar, &s_ok,
-                                        p.status))
-            return;
-    }
-    const float *slam = (OP == OP_GDN) ? s_lamg : reinterpret_cast<const float *>(dsm + lay.lam);
-    float *A = reinterpret_cast<float *>(dsm + lay.A);
-    // Lambda_L per key row: the last snapshot (zero for an empty log)
-    const float *lamL = (L > 0) ? slam + (L - 1) * M : nullptr;
-    {
-        const int AP = up4(L) + 4;
-        for (int idx = tid; idx < DK * (L + 1); idx += NT) {
-            const int i = idx % DK, j = idx / DK;
-            const int x = (OP == OP_GDN) ? 0 : i;
-            const float lL = lamL ? lamL[x] : 0.f;
-            if (j == L)
-                s_gam[i] = expf(lL);
-            else
-                A[i * AP + j] = expf(lL - slam[j * M + x]) * ld_raw(dsm + lay.K, j * DK + i, p.in_bf16);
-        }
+    const float *bh = p.base + (size_t)head * DK * DV + vt * TV + c4;
+    float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
+
+    if (tid < 32) {
+        stage_log<OP, DK, DV, TV>(dsm, lay, p.logK, p.logU, p.logLam, head, vt, L, C, ie, true);
+        cp_async_wait_all();
     }
     __syncthreads();
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
+    for (int x = tid; x < M; x += NT) s_lL[x] = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+    __syncthreads();
+    replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lL, dsm + lay.K, slam, L,
+                             p.in_bf16);
+    __syncthreads();
 
-    const float *tile = reinterpret_cast<const float *>(dsm + lay.tile);
-    float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
+    const float *A = reinterpret_cast<const float *>(dsm + lay.A);
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-#pragma unroll 4
+#pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
         const int row = rg + r * T::RG;
-        const float4 sv = *reinterpret_cast<const float4 *>(tile + row * TV + c4);
-        st_state(dh + (size_t)row * DV, fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
     }
 }
 

@@ -22,11 +22,11 @@ eager_fn get_eager(int op, int dk, int dv);
 // Number of SMs of the current device (cached per device).
 cudaError_t sm_count(int *sms);
 
-// Value-tile width for NH heads of width DV: a whole head per CTA while that
-// still gives at least four CTAs per SM, else the widest tile that does
-// (>= 32 columns).
+// Value-tile width for NH heads of width DV: 64 columns (or the whole head
+// when narrower) while that still gives at least four CTAs per SM, else the
+// widest tile that does (>= 32 columns).
 inline int pick_tile(long long NH, int DV, int sms) {
-    int tv = DV;
+    int tv = DV < 64 ? DV : 64;
     while (tv > 32 && NH * (DV / tv) < 4LL * sms) tv /= 2;
     return tv;
 }

@@ -5,13 +5,12 @@ namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV>
 cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
-    constexpr int NT = (TV == 32) ? 128 : 256;
+    constexpr int NT = 4 * TV;
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = merge_kernel<OP, DK, DV, TV, NT>;
     const int ie = p.in_bf16 ? 2 : 4;
-    const size_t smem = smem_layout<OP, DK, DV, TV, NT>(p.L, ie, false, true, false).bytes;
-    cudaError_t e =
-        allow_smem(smem_ok, kern, smem_layout<OP, DK, DV, TV, NT>(MAXC, 4, false, true, false).bytes);
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, false).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, false).bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)p.NH * (DV / TV);
     kern<<<grid, NT, smem, s>>>(p);

@@ -87,11 +87,6 @@ class DecodeLayer:
     def merge(self, stream=None):
         self.handle.merge(stream)
 
-    def device_status(self) -> int:
-        """The workspace's device-side error bits (0 when all is well)."""
-        _, _, _, oS = B.dl_log_layout(self.cfg)
-        return int(self.log[oS:oS + 4].view(torch.int32).item())
-
     def log_views(self):
         """(K, U, Lambda) views of the log workspace for inspection."""
         oK, oU, oL, _ = B.dl_log_layout(self.cfg)

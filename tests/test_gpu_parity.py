@@ -127,7 +127,6 @@ def test_deltalog_matches_eager_oracle(op, dims, C, mode):
     _, L_ref, _ = oracle.deltalog_run(st, q, k, v, None if op == synth.RWKV6 else beta, g, bon,
                                       w.scale)
     assert Ls == L_ref.tolist()
-    assert layer.device_status() == 0
     o = to_np(outs)
     S = Sr
     for t in range(w.T):
@@ -337,7 +336,6 @@ def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123, mode=B.DL_MERGE
             layer.step(x, t, outs[t])
         mat = layer.materialize()
         torch.cuda.synchronize()
-        assert layer.device_status() == 0
         assert torch.isfinite(outs.float()).all()
         Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, heads=heads, S0=S0, bonus=bonus)
         S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
