@@ -97,20 +97,13 @@ typedef struct dl_handle dl_handle;   /* opaque; host memory only */
  *                                  in_dtype copies of v (RWKV6)
  *   Lambda float [NH, C, m]        cumulative log-decay since the last merge,
  *                                  m = 1 (GDN) or d_k (KDA, RWKV6)
- *   prep   float [NH, P]           per-head results of the ReplayPrep stage of
- *                                  the current token (read-out weights,
- *                                  replay coefficients, decay point); scratch
- *                                  rewritten by every decode step
  * The log is the paper's "bounded update log" (gist.science technical
- * summary, "Meccanismo Core: Base + Log"); the prep area holds what its
- * shared ReplayPrep stage hands to the value-tile AppendDecode stage
- * ("Implementazione del Kernel"). */
+ * summary, "Meccanismo Core: Base + Log"). */
 size_t dl_log_bytes(const dl_config *cfg);
 
-/* Byte offsets of the K, U, Lambda and prep regions of the workspace
- * (any output pointer may be NULL). */
+/* Byte offsets of the K, U and Lambda regions inside the log workspace. */
 dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U,
-                        size_t *off_Lam, size_t *off_prep);
+                        size_t *off_Lam);
 
 /* Create a decode handle over a caller-owned base state (device, fp32
  * [NH, d_k, d_v], 16-byte aligned, holds S at the last merge) and log
@@ -124,8 +117,7 @@ dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,
 
 /* One decode token for all NH heads: the append + read-out step (paper:
  * "Fase di Append", kernel stages ReplayPrep and AppendDecode, gist.science
- * technical summary; two kernels, the second a programmatic dependent launch
- * of the first).  Reads the base once, replays the L logged factors,
+ * technical summary).  Reads the base once, replays the L logged factors,
  * writes `out` (out_dtype [NH, d_v]) and appends (k, u, Lambda) at slot L;
  * the base is not written.  Then L = L + 1.  The token that brings L to C
  * merges: with DL_MERGE_FOLD it is the merge-token (the merged state,

@@ -68,7 +68,7 @@ def lib() -> ctypes.CDLL:
             CP = ctypes.POINTER(dl_config)
             L.dl_log_bytes.argtypes, L.dl_log_bytes.restype = [CP], S
             L.dl_log_layout.argtypes = [CP, ctypes.POINTER(S), ctypes.POINTER(S),
-                                        ctypes.POINTER(S), ctypes.POINTER(S)]
+                                        ctypes.POINTER(S)]
             L.dl_create.argtypes = [CP, P, P, P, ctypes.POINTER(P)]
             L.dl_decode_step.argtypes = [P, P, P, P, P, P, P, P]
             L.dl_merge.argtypes = [P, P]
@@ -128,11 +128,10 @@ def dl_log_bytes(cfg: dl_config) -> int:
 
 
 def dl_log_layout(cfg: dl_config):
-    """(offset of K, of U, of Lambda, of the prep area) in the workspace."""
-    a, b, c, d = (ctypes.c_size_t() for _ in range(4))
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check(lib().dl_log_layout(ctypes.byref(cfg), ctypes.byref(a), ctypes.byref(b),
-                               ctypes.byref(c), ctypes.byref(d)))
-    return a.value, b.value, c.value, d.value
+                               ctypes.byref(c)))
+    return a.value, b.value, c.value
 
 
 def dl_create(cfg: dl_config, base, log_ws, bonus=None) -> int:

@@ -1,31 +1,11 @@
-// append.cu -- launchers of a decode token: ReplayPrep, then AppendDecode
-// (or its merge-token variant) as a programmatic dependent launch.
+// append.cu -- launchers of the append + read-out kernel and its merge-token
+// variant (all ops and shapes).
 #include <mutex>
 
 #include "launch.h"
 
 namespace dl {
 namespace {
-
-// Launch with programmatic stream serialization: the kernel may start while
-// the previous kernel of the stream finishes; it orders itself with
-// griddepcontrol.wait.
-template <typename Kern>
-cudaError_t launch_pdl(Kern kern, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-                       const AppendParams &p) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p);
-}
-
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = 4 * TV;
@@ -35,9 +15,9 @@ cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(replay_prep_kernel<OP, DK, !FOLD>, (unsigned)p.NH, DK, 0, s, p);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(kern, (unsigned)p.NH * (DV / TV), NT, smem, s, p);
+    const unsigned grid = (unsigned)p.NH * (DV / TV);
+    kern<<<grid, NT, smem, s>>>(p);
+    return cudaGetLastError();
 }
 
 template <int OP, int DK, int DV, bool FOLD>

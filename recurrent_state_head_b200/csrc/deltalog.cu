@@ -62,7 +62,7 @@ dl_status check_config(const dl_config *c, bool need_log) {
 }
 
 struct Layout {
-    size_t K, U, Lam, prep, total;
+    size_t K, U, Lam, total;
 };
 
 Layout log_layout(const dl_config *c) {
@@ -73,8 +73,7 @@ Layout log_layout(const dl_config *c) {
     l.K = 0;
     l.U = up256(l.K + nh * C * c->dk * esize(c->in_dtype));
     l.Lam = up256(l.U + nh * C * c->dv * ue);
-    l.prep = up256(l.Lam + nh * C * m * 4);
-    l.total = up256(l.prep + nh * (size_t)dl::prep_stride(c->op, c->dk) * 4);
+    l.total = up256(l.Lam + nh * C * m * 4);
     return l;
 }
 
@@ -135,8 +134,6 @@ dl::AppendParams append_params(const dl_handle *h, const dl_step_io &io, int L) 
     p.scale = h->cfg.scale;
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
     p.out_bf16 = h->cfg.out_dtype == DL_BF16;
-    p.prep = reinterpret_cast<float *>(h->log + h->lay.prep);
-    p.ps = dl::prep_stride(h->cfg.op, h->cfg.dk);
     return p;
 }
 
@@ -175,15 +172,13 @@ size_t dl_log_bytes(const dl_config *cfg) {
     return log_layout(cfg).total;
 }
 
-dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U, size_t *off_Lam,
-                        size_t *off_prep) {
+dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U, size_t *off_Lam) {
     dl_status s = check_config(cfg, true);
     if (s != DL_OK) return s;
     const Layout l = log_layout(cfg);
     if (off_K) *off_K = l.K;
     if (off_U) *off_U = l.U;
     if (off_Lam) *off_Lam = l.Lam;
-    if (off_prep) *off_prep = l.prep;
     return ok();
 }
 

@@ -7,24 +7,14 @@
 // with shared key-side metadata and the ReplayPrep / AppendDecode stages
 // ("Implementazione del Kernel"), operators GDN / KDA / RWKV6.
 //
-// Staged execution, as in the paper: a decode token is two kernels.
-//   ReplayPrep   one CTA per head: the key-side quantities of the token --
-//                decay point, read-out weights, the L replay coefficients and
-//                the self term -- computed once per head into the prep area
-//                of the log workspace; it also appends k_t and Lambda_t to
-//                the log.
-//   AppendDecode one CTA per (head, value tile) (the paper's value-tile
-//                parallelism): streams its tile of the base, reduces S^T w,
-//                replays the log on the value side and writes the output and
-//                u_t.  It is launched as a programmatic dependent of
-//                ReplayPrep: its base loads are issued before it waits for
-//                ReplayPrep's results, so the prep work hides under the base
-//                stream.
-// Tile geometry: TV value columns of all d_k rows, TV/4 threads per row each
-// owning a 16-byte column group, RPT rows per thread held in registers.
-// Nothing here is a dense contraction worth a tensor core: per state element
-// the append does 2 FMAs and the merge at most C = 16, against 4 to 8 bytes
-// of HBM traffic.
+// Decomposition.  A work unit is one head, or one value tile of a head when
+// there are too few heads to fill the GPU (the paper's value-tile split): TV
+// value columns of all d_k rows, so the key-side contractions S^T x reduce
+// inside the CTA.  NT = 4 TV threads: TV/4 threads per row, each owning a
+// 16-byte column group, 16 row groups, RPT = d_k / 16 rows per thread.  The
+// eager kernel always uses 32-column tiles held in registers.  Nothing here is a dense contraction worth a tensor
+// core: per state element the append does 2 FMAs and the merge at most
+// C = 16, against 4 to 8 bytes of HBM traffic.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -48,8 +38,6 @@ struct AppendParams {
     const float *g;           // [NH, m]
     const float *bonus;       // [H, DK]
     void *out;                // [NH, DV] out dtype
-    float *prep;              // [NH, ps] ReplayPrep results (log workspace)
-    int ps;                   // prep stride per head (floats)
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
@@ -145,6 +133,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -200,163 +196,47 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
-// ========================================================= prep layout ==
+// ===================================================== operand staging ==
 //
-// Per-head ReplayPrep results, in floats from the head's prep row:
-//   w     [NA][DK]    read-out weights (Gamma_t * k, Gamma_t * q; RWKV6:
-//                     Gamma_{t-1} * r)
-//   coef  [NA][MAXC]  replay coefficients c_j, d_j (RWKV6: d_j) for j < L
-//   self              k.q (RWKV6: r.(bonus * k))
-//   lt    [M]         Lambda_t (used by the merge-token step)
+// The append, merge-token and merge kernels land everything they read in
+// dynamic shared memory with cp.async, in two copy groups per thread:
+//   group 0  the small operands -- the token's rows, its decay, beta or
+//            bonus, and the L logged entries -- copied by warp 0 alone;
+//   group 1  the base tile, each thread copying the 16-byte chunks it will
+//            itself read back, so the tile needs no barrier.
+// Waiting for group 0 only (cp.async.wait_group 1, a hardware wait) lets the
+// key-side prologue run while the tile is still in flight.  Nothing is held
+// in registers while it travels, so occupancy is bounded by shared memory,
+// and a few CTAs per SM keep enough reads in flight for the HBM rate.
 
 __host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
-template <int OP, int DK>
-struct PrepLayout {
-    static constexpr int M = (OP == OP_GDN) ? 1 : DK;
-    static constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
-    static constexpr int W = 0;
-    static constexpr int COEF = NA * DK;
-    static constexpr int SELF = COEF + NA * MAXC;
-    static constexpr int LT = SELF + 4;
-    static constexpr int HEAD_BYTES = (SELF + 4) * 4;     // w, coef, self: one copy
-    static constexpr int STRIDE = ((LT + M) + 31) / 32 * 32;
-};
-
-// Prep stride (floats per head) for a runtime op / d_k.
-inline int prep_stride(int op, int dk) {
-    const int na = op == OP_RWKV6 ? 1 : 2, m = op == OP_GDN ? 1 : dk;
-    return ((na * dk + na * MAXC + 4 + m) + 31) / 32 * 32;
-}
-
-// ========================================================== ReplayPrep ==
-//
-// One CTA of DK threads per head, thread i owning key channel i:
-//   Lambda_t[i] = Lambda_{L-1}[i] + g_t[i]   (0 before the first entry)
-//   w           = exp(Lambda_t) * k, exp(Lambda_t) * q   (RWKV6: exp(Lambda_{t-1}) * r)
-//   c_j, d_j    = sum_i k_i (q_i) k_j[i] exp(lam_i - Lambda_j[i])  for j < L
-//   self        = k . q   (RWKV6: r . (bonus * k))
-// and, unless this token is a merge-token, the key-side append of k_t and
-// Lambda_t to log slot L.  All loads are issued together (one latency round).
-template <int OP, int DK, bool APPEND>
-__global__ void __launch_bounds__(DK)
-replay_prep_kernel(const AppendParams p) {
-    using PL = PrepLayout<OP, DK>;
-    constexpr int M = PL::M, NA = PL::NA;
-    constexpr int NW = DK / 32;
-    constexpr int NV = NA * MAXC + 1;
-    __shared__ float s_part[NW][NV];
-
-    // let the decode grid launch (it first streams the base), then wait for
-    // the previous kernel of the stream
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
-    const int head = blockIdx.x, i = threadIdx.x;
-    const int lane = i & 31, warp = i >> 5;
-    const int L = p.L, C = p.C;
-    const int x = (OP == OP_GDN) ? 0 : i;
-    const float *lamh = p.logLam + (size_t)head * C * M;
-    const size_t kb = (size_t)head * C * DK + i;
-
-    float kj[MAXC], lj[MAXC];
-#pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-        kj[j] = 0.f;
-        lj[j] = 0.f;
-        if (j < L) {
-            kj[j] = ld_in(p.logK, kb + (size_t)j * DK, p.in_bf16);
-            lj[j] = lamh[j * M + x];
-        }
-    }
-    const float lprev = L > 0 ? lamh[(L - 1) * M + x] : 0.f;
-    const float gi = p.g[(size_t)head * M + x];
-    const float kf = ld_in(p.k, (size_t)head * DK + i, p.in_bf16);
-    const float qf = ld_in(p.q, (size_t)head * DK + i, p.in_bf16);
-    const float bon = (OP == OP_RWKV6) ? p.bonus[(size_t)(head % p.H) * DK + i] : 0.f;
-
-    const float lt = lprev + gi;
-    const float lr = (OP == OP_RWKV6) ? lprev : lt;
-    const float gam = expf(lr);
-    float *pr = p.prep + (size_t)head * p.ps;
-    if (OP == OP_RWKV6) {
-        pr[PL::W + i] = gam * qf;
-    } else {
-        pr[PL::W + i] = gam * kf;
-        pr[PL::W + DK + i] = gam * qf;
-    }
-    if (OP != OP_GDN || i == 0) pr[PL::LT + x] = lt;
-    if (APPEND) {
-        copy_in(p.logK, kb + (size_t)L * DK, p.k, (size_t)head * DK + i, p.in_bf16);
-        if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
-    }
-
-    // per-thread terms of the coefficient dot products, reduced over the CTA
-    float part[NV];
-#pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-        const float e = (OP == OP_GDN) ? kj[j] : expf(lr - lj[j]) * kj[j];
-        if (OP == OP_RWKV6) {
-            part[j] = qf * e;
-        } else {
-            part[j] = kf * e;
-            part[MAXC + j] = qf * e;
-        }
-    }
-    part[NV - 1] = (OP == OP_RWKV6) ? qf * bon * kf : kf * qf;
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-        const int j = v % MAXC;
-        if (v == NV - 1 || j < L) {
-            const float s = warp_sum(part[v]);
-            if (lane == 0) s_part[warp][v] = s;
-        }
-    }
-    __syncthreads();
-    for (int v = i; v < NV; v += DK) {
-        const int j = v % MAXC;
-        if (v != NV - 1 && j >= L) continue;
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) s += s_part[w][v];
-        if (OP == OP_GDN && v != NV - 1) s *= expf(lt - lamh[j]);   // scalar decay of entry j
-        pr[PL::COEF + v] = s;                                      // coef[a][j] and self
-    }
-}
-
-// ===================================================== operand staging ==
-//
-// The decode, merge-token and merge kernels hold their base tile in
-// registers (16-byte loads issued first) and stage the small operands in
-// dynamic shared memory with cp.async issued by warp 0 alone, waited for
-// with cp.async.wait_all (a hardware wait) and published with __syncthreads.
-
 // Byte offsets of the staged operands (all 16-byte aligned).
 struct OpLayout {
-    int prep, lt, kin, vin, beta, K, lam, U, A, bytes;
+    int tile, kin, qin, vin, g, beta, bonus, K, lam, U, A, bytes;
 };
 
-// decode: the head's prep row (w, coef, self), v tile, beta, the tile's L
-// value factors.  fold adds Lambda_t, k and the L logged keys and decay
-// snapshots, and the [DK][up4(L) + 4] replay-factor table.  merge: the log
-// entries and the table only.
+// tile: the [DK][TV] fp32 base tile.  token: the token's k, q (r), v tile,
+// g, beta / bonus.  A: room for the [DK][up4(L) + 4] fp32 table of per-row
+// replay factors (merge, merge-token).
 template <int OP, int DK, int TV>
-__host__ __device__ inline OpLayout op_layout(int L, int ie, bool decode, bool fold) {
-    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+__host__ __device__ inline OpLayout op_layout(int L, int ie, bool token, bool table) {
+    const int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
-    const bool logkeys = fold || !decode;
     OpLayout s{};
     int o = 0;
-    s.prep = o; o += decode ? PrepLayout<OP, DK>::HEAD_BYTES : 0;
-    s.lt = o; o += fold ? up16(M * 4) : 0;
-    s.kin = o; o += fold ? up16(DK * ie) : 0;
-    s.vin = o; o += decode ? up16(TV * ie) : 0;
-    s.beta = o; o += decode ? 16 : 0;
-    s.K = o; o += logkeys ? up16(L * DK * ie) : 0;
-    s.lam = o; o += logkeys ? up16(L * M * 4) : 0;
+    s.tile = o; o += DK * TV * 4;
+    s.kin = o; o += token ? up16(DK * ie) : 0;
+    s.qin = o; o += token ? up16(DK * ie) : 0;
+    s.vin = o; o += token ? up16(TV * ie) : 0;
+    s.g = o; o += token ? up16(M * 4) : 0;
+    s.beta = o; o += token ? 16 : 0;
+    s.bonus = o; o += (token && OP == OP_RWKV6) ? DK * 4 : 0;
+    s.K = o; o += up16(L * DK * ie);
+    s.lam = o; o += up16(L * M * 4);
     s.U = o; o += up16(L * TV * ue);
-    s.A = o; o += logkeys ? DK * (up4(L) + 4) * 4 : 0;
+    s.A = o; o += table ? DK * (up4(L) + 4) * 4 : 0;
     s.bytes = o;
     return s;
 }
@@ -367,25 +247,45 @@ __device__ __forceinline__ void warp_copy(unsigned char *dst, const void *src, i
     for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, g + o);
 }
 
-// Stage the L logged entries of one head / value tile (warp 0).
+// Sources of one head's staged operands.
+struct OpSources {
+    const void *k, *q, *v;          // token rows (NULL: not staged)
+    const float *g, *beta, *bonus;
+    const void *logK, *logU;
+    const float *logLam;
+};
+
+// Stage one unit's small operands (warp 0 only; the caller commits the group).
 template <int OP, int DK, int DV, int TV>
-__device__ __forceinline__ void stage_log(unsigned char *sm, const OpLayout &lay, const void *logK,
-                                          const void *logU, const float *logLam, int head, int vt, int L,
-                                          int C, int ie, bool keys) {
+__device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay, const OpSources &src,
+                                          int head, int vt, int L, int C, int H, int ie, bool token) {
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
     const int lane = threadIdx.x & 31;
-    if (keys) {
-        warp_copy(sm + lay.K, static_cast<const char *>(logK) + (size_t)head * C * DK * ie, L * DK * ie,
-                  lane);
-        const float *lamh = logLam + (size_t)head * C * M;
+    if (token) {
+        warp_copy(sm + lay.kin, static_cast<const char *>(src.k) + (size_t)head * DK * ie, DK * ie, lane);
+        warp_copy(sm + lay.qin, static_cast<const char *>(src.q) + (size_t)head * DK * ie, DK * ie, lane);
+        warp_copy(sm + lay.vin, static_cast<const char *>(src.v) + ((size_t)head * DV + vt * TV) * ie,
+                  TV * ie, lane);
         if (OP == OP_GDN) {
-            for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
+            if (lane == 0) cp_async4(sm + lay.g, src.g + head);
         } else {
-            warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
+            warp_copy(sm + lay.g, src.g + (size_t)head * DK, DK * 4, lane);
         }
+        if (OP == OP_RWKV6)
+            warp_copy(sm + lay.bonus, src.bonus + (size_t)(head % H) * DK, DK * 4, lane);
+        else if (lane == 1)
+            cp_async4(sm + lay.beta, src.beta + head);
     }
-    const char *lU = static_cast<const char *>(logU) + ((size_t)head * C * DV + vt * TV) * ue;
+    warp_copy(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie, L * DK * ie,
+              lane);
+    const float *lamh = src.logLam + (size_t)head * C * M;
+    if (OP == OP_GDN) {
+        for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
+    } else {
+        warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
+    }
+    const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
     const int cpr = TV * ue / 16;
     for (int idx = lane; idx < L * cpr; idx += 32) {
         const int j = idx / cpr, c = idx - j * cpr;
@@ -421,7 +321,7 @@ __device__ __forceinline__ void replay_table(float *A, float *gam, const float *
     }
 }
 
-// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3]
+// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3] (+ kr * w4)
 template <int TV>
 __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow, const unsigned char *sU,
                                            int c4, int L, int ubf) {
@@ -443,30 +343,42 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
     return o;
 }
 
-// ======================================== AppendDecode (+ merge-token) ==
+// ============================================ append + read-out (+ fold) ==
 //
-// One CTA per (head, value tile), after ReplayPrep: x = Sbar^T w over the
-// register tile (the one base read), value-side replay r = sum_j coef_j u_j,
-// delta correction u = beta (v - x_k - r_k), output o = scale (x_q + r_q +
-// self u) (RWKV6: o = scale (x_r + r_r + self v)).
-// FOLD = false (append, "Fase di Append"): u_t goes to log slot L; the base
-//   is not written.
-// FOLD = true (merge-token, the token that completes the log: "Fase di
+// One CTA per unit (a head, or a TV-column value tile of a head).
+// ReplayPrep (once per CTA): decay point Lambda_t = Lambda_{L-1} + g_t
+// (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
+// Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
+// (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
+// x = Sbar^T w over the register tile (the one base read), value-side replay,
+// delta correction, output.
+// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
+//   slot L; the base is not written.
+// FOLD = true (merge-token, the step that completes the log: "Fase di
 //   Merge"): the logical state after this token -- base decayed to Lambda_t,
 //   all L logged factors and this token's k u^T -- is written over the base
-//   tile (read once, written once); the caller resets the log (L = 0).
+//   tile (the register tile is read once and written once); the log is left
+//   for the caller to reset (L = 0).
 template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
-    using PL = PrepLayout<OP, DK>;
-    constexpr int NA = PL::NA;
+    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
     extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ float s_lt[DK];           // Lambda_t
+    __shared__ float s_lr[DK];           // decay point of read-out and replay
+    __shared__ float s_k[DK];
+    __shared__ float s_q[DK];
+    __shared__ float s_w[NA][DK];        // read-out weights
+    __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
+    __shared__ float s_gam[FOLD ? DK : 1];
+    __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
+    __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
     __shared__ __align__(16) float s_red[NA * T::NW * TV];
     __shared__ float s_x[NA * TV];
-    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
     const int unit = blockIdx.x;
@@ -478,44 +390,92 @@ append_kernel(const AppendParams p) {
     const int c4 = col4 * 4;
     const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
 
-    // 1. the base stream: RPT rows x 16 bytes per thread (independent of
-    //    ReplayPrep, so it starts before waiting for it)
+    // 1. small operands (warp 0, copy group 0), then the base tile: RPT rows
+    //    x 16 bytes per thread, each thread copying what it reads (group 1)
+    if (tid < 32) {
+        const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true);
+    }
+    cp_async_commit();
     float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
-    float4 s[T::RPT];
+    unsigned char *tl = dsm + lay.tile + c4 * 4;
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r)
-        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
-                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+        cp_async16(tl + (rg + r * T::RG) * TV * 4, bh + (size_t)(rg + r * T::RG) * DV);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
 
-    // 2. ReplayPrep's results and the value-side operands
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid < 32) {
-        const int lane = tid;
-        warp_copy(dsm + lay.prep, p.prep + (size_t)head * p.ps, PL::HEAD_BYTES, lane);
-        warp_copy(dsm + lay.vin, static_cast<const char *>(p.v) + ((size_t)head * DV + vt * TV) * ie,
-                  TV * ie, lane);
-        if (OP != OP_RWKV6 && lane == 0) cp_async4(dsm + lay.beta, p.beta + head);
-        if (FOLD) {
-            if (OP == OP_GDN) {
-                if (lane == 1) cp_async4(dsm + lay.lt, p.prep + (size_t)head * p.ps + PL::LT);
-            } else {
-                warp_copy(dsm + lay.lt, p.prep + (size_t)head * p.ps + PL::LT, DK * 4, lane);
-            }
-            warp_copy(dsm + lay.kin, static_cast<const char *>(p.k) + (size_t)head * DK * ie, DK * ie, lane);
+    // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
+    if (tid < DK) {
+        const int i = tid;
+        const int x = (OP == OP_GDN) ? 0 : i;
+        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+        const float lt = lprev + sg[x];
+        const float lr = (OP == OP_RWKV6) ? lprev : lt;
+        const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
+        const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
+        const float gam = expf(lr);
+        s_lt[i] = lt;
+        s_lr[i] = lr;
+        s_k[i] = kf;
+        s_q[i] = qf;
+        if (OP == OP_RWKV6) {
+            s_w[0][i] = gam * qf;
+            s_bk[i] = reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf;
+        } else {
+            s_w[0][i] = gam * kf;
+            s_w[NA - 1][i] = gam * qf;
         }
-        stage_log<OP, DK, DV, TV>(dsm, lay, p.logK, p.logU, p.logLam, head, vt, L, C, ie, FOLD);
-        cp_async_wait_all();
+        if (!FOLD && vt == 0) {
+            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
+            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
+        }
     }
     __syncthreads();
-    const float *sp = reinterpret_cast<const float *>(dsm + lay.prep);
-    if (FOLD) {
-        replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam,
-                                 reinterpret_cast<const float *>(dsm + lay.lt), dsm + lay.K,
-                                 reinterpret_cast<const float *>(dsm + lay.lam), L, p.in_bf16);
-        __syncthreads();
-    }
 
-    // 3. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    // replay coefficients: task tau < L is log entry tau, tau == L the self term
+    {
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int tau = warp; tau <= L; tau += T::NW) {
+            float a0 = 0.f, a1 = 0.f;
+            if (tau < L) {
+                const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
+#pragma unroll
+                for (int i = lane; i < DK; i += 32) {
+                    const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
+                    const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
+                    if (OP == OP_RWKV6) {
+                        a0 = fmaf(s_q[i], e, a0);
+                    } else {
+                        a0 = fmaf(s_k[i], e, a0);
+                        a1 = fmaf(s_q[i], e, a1);
+                    }
+                }
+                a0 = warp_sum(a0) * gdec;
+                if (NA == 2) a1 = warp_sum(a1) * gdec;
+                if (lane == 0) {
+                    s_coef[0][tau] = a0;
+                    if (NA == 2) s_coef[NA - 1][tau] = a1;
+                }
+            } else {
+#pragma unroll
+                for (int i = lane; i < DK; i += 32)
+                    a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
+                a0 = warp_sum(a0);
+                if (lane == 0) s_self = a0;
+            }
+        }
+    }
+    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
+                                       dsm + lay.K, slam, L, p.in_bf16);
+    __syncthreads();
+
+    // 4. base read-out from this thread's own staged chunks:
+    //    x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    cp_async_wait_group<0>();
     {
         float4 acc[NA];
 #pragma unroll
@@ -523,30 +483,30 @@ append_kernel(const AppendParams p) {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
+            const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
-                const float w = sp[PL::W + a * DK + row];
-                acc[a].x = fmaf(w, s[r].x, acc[a].x);
-                acc[a].y = fmaf(w, s[r].y, acc[a].y);
-                acc[a].z = fmaf(w, s[r].z, acc[a].z);
-                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+                const float w = s_w[a][row];
+                acc[a].x = fmaf(w, sv.x, acc[a].x);
+                acc[a].y = fmaf(w, sv.y, acc[a].y);
+                acc[a].z = fmaf(w, sv.z, acc[a].z);
+                acc[a].w = fmaf(w, sv.w, acc[a].w);
             }
         }
         reduce_rows<NA, TV, NT>(acc, s_red, s_x);
     }
 
-    // 4. value side: log replay, delta correction, output, append of u
+    // 5. value side: log replay, delta correction, output, append of u
     if (tid < TV) {
         const int c = tid;
         const int col = vt * TV + c;
         const size_t ub = (size_t)head * C * DV + col;
         const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
-        const float *cf = sp + PL::COEF;
-        const float self = sp[PL::SELF];
         if (OP == OP_RWKV6) {
             float rr = 0.f;
-            for (int j = 0; j < L; ++j) rr = fmaf(cf[j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
-            const float o = p.scale * (s_x[c] + rr + self * vv);
+            for (int j = 0; j < L; ++j)
+                rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
+            const float o = p.scale * (s_x[c] + rr + s_self * vv);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = vv;
@@ -557,12 +517,12 @@ append_kernel(const AppendParams p) {
             float rk = 0.f, rq = 0.f;
             for (int j = 0; j < L; ++j) {
                 const float uj = U[j * TV + c];
-                rk = fmaf(cf[j], uj, rk);
-                rq = fmaf(cf[MAXC + j], uj, rq);
+                rk = fmaf(s_coef[0][j], uj, rk);
+                rq = fmaf(s_coef[1][j], uj, rq);
             }
             const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
             const float u = beta * (vv - s_x[c] - rk);
-            const float o = p.scale * (s_x[TV + c] + rq + self * u);
+            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = u;
@@ -571,7 +531,7 @@ append_kernel(const AppendParams p) {
         }
     }
 
-    // 5. merge-token: write the logical state after this token over the base
+    // 6. merge-token: write the logical state after this token over the base
     if (FOLD) {
         __syncthreads();
         const float *A = reinterpret_cast<const float *>(dsm + lay.A);
@@ -581,8 +541,9 @@ append_kernel(const AppendParams p) {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
-            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-            const float kr = ld_raw(dsm + lay.kin, row, p.in_bf16);
+            const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
+            float4 o = fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+            const float kr = s_k[row];
             o.x = fmaf(kr, u4.x, o.x);
             o.y = fmaf(kr, u4.y, o.y);
             o.z = fmaf(kr, u4.z, o.z);
@@ -616,18 +577,21 @@ merge_kernel(const MergeParams p) {
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, false, false);
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, false, true);
 
     const float *bh = p.base + (size_t)head * DK * DV + vt * TV + c4;
     float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
-    float4 s[T::RPT];
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
-
     if (tid < 32) {
-        stage_log<OP, DK, DV, TV>(dsm, lay, p.logK, p.logU, p.logLam, head, vt, L, C, ie, true);
-        cp_async_wait_all();
+        const OpSources src{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false);
     }
+    cp_async_commit();
+    unsigned char *tl = dsm + lay.tile + c4 * 4;
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r)
+        cp_async16(tl + (rg + r * T::RG) * TV * 4, bh + (size_t)(rg + r * T::RG) * DV);
+    cp_async_commit();
+    cp_async_wait_group<1>();
     __syncthreads();
     const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
     for (int x = tid; x < M; x += NT) s_lL[x] = L > 0 ? slam[(L - 1) * M + x] : 0.f;
@@ -639,10 +603,12 @@ merge_kernel(const MergeParams p) {
     const float *A = reinterpret_cast<const float *>(dsm + lay.A);
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+    cp_async_wait_group<0>();
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
         const int row = rg + r * T::RG;
-        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
+        st_state(dh + (size_t)row * DV, fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
     }
 }
 

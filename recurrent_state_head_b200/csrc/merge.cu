@@ -9,8 +9,8 @@ cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = merge_kernel<OP, DK, DV, TV, NT>;
     const int ie = p.in_bf16 ? 2 : 4;
-    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, false).bytes;
-    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, false).bytes);
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, true).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, true).bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)p.NH * (DV / TV);
     kern<<<grid, NT, smem, s>>>(p);

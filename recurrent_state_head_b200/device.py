@@ -89,7 +89,7 @@ class DecodeLayer:
 
     def log_views(self):
         """(K, U, Lambda) views of the log workspace for inspection."""
-        oK, oU, oL, _ = B.dl_log_layout(self.cfg)
+        oK, oU, oL = B.dl_log_layout(self.cfg)
         NH, C, dk, dv, m = self.w.heads, self.cfg.C, self.w.dk, self.w.dv, self.w.m
         in_t = TORCH_DTYPE[self.w.in_dtype]
         u_t = in_t if self.w.op == RWKV6 else torch.float32
