@@ -345,20 +345,25 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
 
 // ============================================ append + read-out (+ fold) ==
 //
-// One CTA per unit (a head, or a TV-column value tile of a head).
-// ReplayPrep (once per CTA): decay point Lambda_t = Lambda_{L-1} + g_t
-// (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
-// Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
-// (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
-// x = Sbar^T w over the register tile (the one base read), value-side replay,
-// delta correction, output.
-// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
-//   slot L; the base is not written.
-// FOLD = true (merge-token, the step that completes the log: "Fase di
+// One CTA per unit (a head, or a TV-column value tile of a head), two CTA
+// barriers in all:
+//   staging    small operands (warp 0) and the base tile (every thread, its
+//              own chunks) land in shared memory; barrier 1
+//   per warp   ReplayPrep: the warp's share of the replay coefficients
+//              c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]} (d_j with q) and
+//              the self term k.q (RWKV6: r.(bonus*k)); then AppendDecode on
+//              its rows: read-out weights Gamma * k, Gamma * q (RWKV6:
+//              Gamma_{t-1} * r) for each row it owns, x = Sbar^T w partial
+//              sums, folded across the warp's row groups; barrier 2
+//   epilogue   the TV column threads finish x, replay the log on the value
+//              side, apply the delta correction and write the output.
+// Lambda_t = Lambda_{L-1} + g_t (RWKV6 reads at Lambda_{t-1}).
+// FOLD = false (append, "Fase di Append"): u_t, and (first tile of each
+//   head) k_t and Lambda_t, go to log slot L; the base is not written.
+// FOLD = true (merge-token, the token that completes the log: "Fase di
 //   Merge"): the logical state after this token -- base decayed to Lambda_t,
 //   all L logged factors and this token's k u^T -- is written over the base
-//   tile (the register tile is read once and written once); the log is left
-//   for the caller to reset (L = 0).
+//   tile (read once, written once); the caller resets the log (L = 0).
 template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
@@ -368,22 +373,15 @@ append_kernel(const AppendParams p) {
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
 
     extern __shared__ __align__(16) unsigned char dsm[];
-    __shared__ float s_lt[DK];           // Lambda_t
-    __shared__ float s_lr[DK];           // decay point of read-out and replay
-    __shared__ float s_k[DK];
-    __shared__ float s_q[DK];
-    __shared__ float s_w[NA][DK];        // read-out weights
-    __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
-    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
-    __shared__ __align__(16) float s_red[NA * T::NW * TV];
-    __shared__ float s_x[NA * TV];
+    __shared__ __align__(16) float s_red[T::NW][NA][TV];   // per-warp row partials
+    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
     const int unit = blockIdx.x;
     const int head = unit / T::NVT, vt = unit - head * T::NVT;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = p.L, C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
@@ -404,79 +402,67 @@ append_kernel(const AppendParams p) {
         cp_async16(tl + (rg + r * T::RG) * TV * 4, bh + (size_t)(rg + r * T::RG) * DV);
     cp_async_commit();
     cp_async_wait_group<1>();
-    __syncthreads();
+    __syncthreads();                                        // barrier 1
+
     const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
     const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
-
-    // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
-    if (tid < DK) {
-        const int i = tid;
+    const unsigned char *skin = dsm + lay.kin, *sqin = dsm + lay.qin;
+    // decay point of key channel i: Lambda_t (RWKV6: Lambda_{t-1})
+    auto lam_r = [&](int i) {
         const int x = (OP == OP_GDN) ? 0 : i;
         const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-        const float lt = lprev + sg[x];
-        const float lr = (OP == OP_RWKV6) ? lprev : lt;
-        const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
-        const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
-        const float gam = expf(lr);
-        s_lt[i] = lt;
-        s_lr[i] = lr;
-        s_k[i] = kf;
-        s_q[i] = qf;
-        if (OP == OP_RWKV6) {
-            s_w[0][i] = gam * qf;
-            s_bk[i] = reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf;
-        } else {
-            s_w[0][i] = gam * kf;
-            s_w[NA - 1][i] = gam * qf;
-        }
-        if (!FOLD && vt == 0) {
-            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
-            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
-        }
-    }
-    __syncthreads();
+        return (OP == OP_RWKV6) ? lprev : lprev + sg[x];
+    };
 
-    // replay coefficients: task tau < L is log entry tau, tau == L the self term
-    {
-        const int lane = tid & 31, warp = tid >> 5;
-        for (int tau = warp; tau <= L; tau += T::NW) {
-            float a0 = 0.f, a1 = 0.f;
-            if (tau < L) {
-                const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
+    // 2a. key-side append of k_t and Lambda_t (first tile of the head)
+    if (!FOLD && vt == 0 && tid < DK) {
+        const int i = tid, x = (OP == OP_GDN) ? 0 : i;
+        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+        copy_raw(p.logK, ((size_t)head * C + L) * DK + i, skin, i, p.in_bf16);
+        if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lprev + sg[x];
+    }
+
+    // 2b. ReplayPrep, this warp's share: task tau < L is log entry tau,
+    //     tau == L the self term
+    for (int tau = warp; tau <= L; tau += T::NW) {
+        float a0 = 0.f, a1 = 0.f;
+        if (tau < L) {
+            const float gdec = (OP == OP_GDN) ? expf(lam_r(0) - slam[tau]) : 1.f;
 #pragma unroll
-                for (int i = lane; i < DK; i += 32) {
-                    const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
-                    const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
-                    if (OP == OP_RWKV6) {
-                        a0 = fmaf(s_q[i], e, a0);
-                    } else {
-                        a0 = fmaf(s_k[i], e, a0);
-                        a1 = fmaf(s_q[i], e, a1);
-                    }
+            for (int i = lane; i < DK; i += 32) {
+                const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
+                const float e = (OP == OP_GDN) ? kj : expf(lam_r(i) - slam[tau * M + i]) * kj;
+                const float qf = ld_raw(sqin, i, p.in_bf16);
+                if (OP == OP_RWKV6) {
+                    a0 = fmaf(qf, e, a0);
+                } else {
+                    a0 = fmaf(ld_raw(skin, i, p.in_bf16), e, a0);
+                    a1 = fmaf(qf, e, a1);
                 }
-                a0 = warp_sum(a0) * gdec;
-                if (NA == 2) a1 = warp_sum(a1) * gdec;
-                if (lane == 0) {
-                    s_coef[0][tau] = a0;
-                    if (NA == 2) s_coef[NA - 1][tau] = a1;
-                }
-            } else {
-#pragma unroll
-                for (int i = lane; i < DK; i += 32)
-                    a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
-                a0 = warp_sum(a0);
-                if (lane == 0) s_self = a0;
             }
+            a0 = warp_sum(a0) * gdec;
+            if (NA == 2) a1 = warp_sum(a1) * gdec;
+            if (lane == 0) {
+                s_coef[0][tau] = a0;
+                if (NA == 2) s_coef[NA - 1][tau] = a1;
+            }
+        } else {
+            const float *sbon = reinterpret_cast<const float *>(dsm + lay.bonus);
+#pragma unroll
+            for (int i = lane; i < DK; i += 32) {
+                const float kf = ld_raw(skin, i, p.in_bf16), qf = ld_raw(sqin, i, p.in_bf16);
+                a0 = fmaf(qf, (OP == OP_RWKV6) ? sbon[i] * kf : kf, a0);
+            }
+            a0 = warp_sum(a0);
+            if (lane == 0) s_self = a0;
         }
     }
-    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
-                                       dsm + lay.K, slam, L, p.in_bf16);
-    __syncthreads();
 
-    // 4. base read-out from this thread's own staged chunks:
-    //    x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    // 2c. AppendDecode on this thread's rows of the staged tile:
+    //     x_a[c] = sum_i w_a[i] * Sbar[i][c], weights formed per row
     cp_async_wait_group<0>();
     {
+        const float gsc = (OP == OP_GDN) ? expf(lam_r(0)) : 1.f;
         float4 acc[NA];
 #pragma unroll
         for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -484,29 +470,55 @@ append_kernel(const AppendParams p) {
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
             const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
+            const float gam = (OP == OP_GDN) ? gsc : expf(lam_r(row));
+            float w[NA];
+            if (OP == OP_RWKV6) {
+                w[0] = gam * ld_raw(sqin, row, p.in_bf16);
+            } else {
+                w[0] = gam * ld_raw(skin, row, p.in_bf16);
+                w[NA - 1] = gam * ld_raw(sqin, row, p.in_bf16);
+            }
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
-                const float w = s_w[a][row];
-                acc[a].x = fmaf(w, sv.x, acc[a].x);
-                acc[a].y = fmaf(w, sv.y, acc[a].y);
-                acc[a].z = fmaf(w, sv.z, acc[a].z);
-                acc[a].w = fmaf(w, sv.w, acc[a].w);
+                acc[a].x = fmaf(w[a], sv.x, acc[a].x);
+                acc[a].y = fmaf(w[a], sv.y, acc[a].y);
+                acc[a].z = fmaf(w[a], sv.z, acc[a].z);
+                acc[a].w = fmaf(w[a], sv.w, acc[a].w);
             }
         }
-        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
+        // fold the warp's row groups, then one row of partials per warp
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+#pragma unroll
+            for (int o = T::TPR; o < 32; o <<= 1) {
+                acc[a].x += __shfl_xor_sync(0xffffffffu, acc[a].x, o);
+                acc[a].y += __shfl_xor_sync(0xffffffffu, acc[a].y, o);
+                acc[a].z += __shfl_xor_sync(0xffffffffu, acc[a].z, o);
+                acc[a].w += __shfl_xor_sync(0xffffffffu, acc[a].w, o);
+            }
+            if (lane < T::TPR) *reinterpret_cast<float4 *>(&s_red[warp][a][c4]) = acc[a];
+        }
     }
+    __syncthreads();                                        // barrier 2
 
-    // 5. value side: log replay, delta correction, output, append of u
+    // 3. value side: finish x, log replay, delta correction, output, append of u
     if (tid < TV) {
         const int c = tid;
         const int col = vt * TV + c;
         const size_t ub = (size_t)head * C * DV + col;
+        float x[NA];
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < T::NW; ++w) sum += s_red[w][a][c];
+            x[a] = sum;
+        }
         const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
         if (OP == OP_RWKV6) {
             float rr = 0.f;
-            for (int j = 0; j < L; ++j)
-                rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
-            const float o = p.scale * (s_x[c] + rr + s_self * vv);
+            for (int j = 0; j < L; ++j) rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
+            const float o = p.scale * (x[0] + rr + s_self * vv);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = vv;
@@ -521,8 +533,8 @@ append_kernel(const AppendParams p) {
                 rq = fmaf(s_coef[1][j], uj, rq);
             }
             const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
-            const float u = beta * (vv - s_x[c] - rk);
-            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+            const float u = beta * (vv - x[0] - rk);
+            const float o = p.scale * (x[NA - 1] + rq + s_self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = u;
@@ -531,10 +543,24 @@ append_kernel(const AppendParams p) {
         }
     }
 
-    // 6. merge-token: write the logical state after this token over the base
+    // 4. merge-token: write the logical state after this token over the base
     if (FOLD) {
+        // replay-factor table with Lambda_t, then the new rows
+        float *A = reinterpret_cast<float *>(dsm + lay.A);
+        {
+            const int AP = up4(L) + 4;
+            for (int idx = tid; idx < DK * (L + 1); idx += NT) {
+                const int i = idx % DK, j = idx / DK;
+                const int x = (OP == OP_GDN) ? 0 : i;
+                const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+                const float lt = lprev + sg[x];
+                if (j == L)
+                    s_gam[i] = expf(lt);
+                else
+                    A[i * AP + j] = expf(lt - slam[j * M + x]) * ld_raw(dsm + lay.K, j * DK + i, p.in_bf16);
+            }
+        }
         __syncthreads();
-        const float *A = reinterpret_cast<const float *>(dsm + lay.A);
         const int AP = up4(L) + 4;
         const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
         const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
@@ -543,7 +569,7 @@ append_kernel(const AppendParams p) {
             const int row = rg + r * T::RG;
             const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
             float4 o = fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-            const float kr = s_k[row];
+            const float kr = ld_raw(skin, row, p.in_bf16);
             o.x = fmaf(kr, u4.x, o.x);
             o.y = fmaf(kr, u4.y, o.y);
             o.z = fmaf(kr, u4.z, o.z);
