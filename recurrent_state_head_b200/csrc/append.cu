@@ -1,6 +1,5 @@
 // append.cu -- launchers of the append + read-out kernel and its merge-token
 // variant (all ops and shapes).
-#include <algorithm>
 #include <mutex>
 
 #include "launch.h"
@@ -8,20 +7,15 @@
 namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV, bool FOLD>
-cudaError_t launch_tv(const AppendParams &p, cudaStream_t s, int sms) {
-    constexpr int NT = 4 * TV, NS = Pipe<TV>::NS;
+cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
+    constexpr int NT = 4 * TV;
     static std::atomic<unsigned long long> smem_ok{0};
-    static OccupancyCache occ;
-    auto kern = append_kernel<OP, DK, DV, TV, NT, NS, FOLD>;
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD>;
     const int ie = p.in_bf16 ? 2 : 4;
-    const size_t smem = (size_t)NS * up16(op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes);
-    cudaError_t e =
-        allow_smem(smem_ok, kern, (size_t)NS * up16(op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes));
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    if ((e = occ.get(kern, NT, smem, &per_sm)) != cudaSuccess) return e;
-    const long long units = (long long)p.NH * (DV / TV);
-    const unsigned grid = (unsigned)std::min<long long>(units, (long long)sms * per_sm);
+    const unsigned grid = (unsigned)p.NH * (DV / TV);
     kern<<<grid, NT, smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -32,11 +26,11 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
     cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
     switch (pick_tile(p.NH, DV, sms)) {
-        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, FOLD>(p, s, sms); break;
-        case 64: return launch_tv<OP, DK, DV, 64, FOLD>(p, s, sms);
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, FOLD>(p, s); break;
+        case 64: return launch_tv<OP, DK, DV, 64, FOLD>(p, s);
         default: break;
     }
-    return launch_tv<OP, DK, DV, 32, FOLD>(p, s, sms);
+    return launch_tv<OP, DK, DV, 32, FOLD>(p, s);
 }
 
 template <int OP, int DK, int DV>

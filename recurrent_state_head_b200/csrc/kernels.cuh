@@ -11,8 +11,8 @@
 // there are too few heads to fill the GPU (the paper's value-tile split): TV
 // value columns of all d_k rows, so the key-side contractions S^T x reduce
 // inside the CTA.  NT = 4 TV threads: TV/4 threads per row, each owning a
-// 16-byte column group, 16 row groups, RPT = d_k / 16 rows per thread.  The
-// eager kernel always uses 32-column tiles held in registers.  Nothing here is a dense contraction worth a tensor
+// 16-byte column group, 16 row groups, RPT = d_k / 16 rows per thread held in
+// registers.  The eager kernel always uses 32-column tiles.  Nothing here is a dense contraction worth a tensor
 // core: per state element the append does 2 FMAs and the merge at most
 // C = 16, against 4 to 8 bytes of HBM traffic.
 #pragma once
@@ -133,14 +133,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-// Wait until at most N of this thread's committed copy groups are pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -198,35 +190,30 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
 
 // ===================================================== operand staging ==
 //
-// The append, merge-token and merge kernels land everything they read in
-// dynamic shared memory with cp.async, in two copy groups per thread:
-//   group 0  the small operands -- the token's rows, its decay, beta or
-//            bonus, and the L logged entries -- copied by warp 0 alone;
-//   group 1  the base tile, each thread copying the 16-byte chunks it will
-//            itself read back, so the tile needs no barrier.
-// Waiting for group 0 only (cp.async.wait_group 1, a hardware wait) lets the
-// key-side prologue run while the tile is still in flight.  Nothing is held
-// in registers while it travels, so occupancy is bounded by shared memory,
-// and a few CTAs per SM keep enough reads in flight for the HBM rate.
+// The append, merge-token and merge kernels hold their base tile in
+// registers (16-byte loads issued first, so they are in flight while
+// everything else happens) and stage the small operands -- the token's rows,
+// its decay, beta or bonus, and the L logged entries -- in dynamic shared
+// memory with cp.async issued by warp 0 alone, waited for with
+// cp.async.wait_all (a hardware wait) and published with __syncthreads.
 
 __host__ __device__ constexpr int up16(int x) { return (x + 15) & ~15; }
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
 // Byte offsets of the staged operands (all 16-byte aligned).
 struct OpLayout {
-    int tile, kin, qin, vin, g, beta, bonus, K, lam, U, A, bytes;
+    int kin, qin, vin, g, beta, bonus, K, lam, U, A, bytes;
 };
 
-// tile: the [DK][TV] fp32 base tile.  token: the token's k, q (r), v tile,
-// g, beta / bonus.  A: room for the [DK][up4(L) + 4] fp32 table of per-row
-// replay factors (merge, merge-token).
+// token: stage the token's k, q (r), v tile, g, beta / bonus.  A: room for
+// the [DK][up4(L) + 4] fp32 table of per-row replay factors (merge,
+// merge-token).
 template <int OP, int DK, int TV>
 __host__ __device__ inline OpLayout op_layout(int L, int ie, bool token, bool table) {
     const int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
     OpLayout s{};
     int o = 0;
-    s.tile = o; o += DK * TV * 4;
     s.kin = o; o += token ? up16(DK * ie) : 0;
     s.qin = o; o += token ? up16(DK * ie) : 0;
     s.vin = o; o += token ? up16(TV * ie) : 0;
@@ -255,7 +242,7 @@ struct OpSources {
     const float *logLam;
 };
 
-// Stage one unit's small operands (warp 0 only; the caller commits the group).
+// Stage one unit's operands (warp 0 only), then wait for them.
 template <int OP, int DK, int DV, int TV>
 __device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay, const OpSources &src,
                                           int head, int vt, int L, int C, int H, int ie, bool token) {
@@ -291,6 +278,7 @@ __device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay
         const int j = idx / cpr, c = idx - j * cpr;
         cp_async16(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16);
     }
+    cp_async_wait_all();
 }
 
 // Four consecutive elements of a raw vector in shared memory as fp32.
@@ -345,127 +333,112 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
 
 // ============================================ append + read-out (+ fold) ==
 //
-// Persistent: a grid of (SM count x resident CTAs per SM) CTAs walks the
-// units (a head, or a TV-column value tile of a head) with a stride of
-// gridDim.x.  Each unit's operands form one stage of dynamic shared memory;
-// NS stages rotate, so while a unit runs its phases the tiles and operands
-// of the next NS-1 units are already streaming in.  A stage is filled by two
-// kinds of cp.async: the small operands (the token's rows, decay, beta or
-// bonus, and the L logged entries) by warp 0, and the base tile by every
-// thread, each copying the 16-byte chunks it will read back itself.
-// Per unit, two CTA barriers:
-//   barrier 1  the unit's stage has landed
-//   per warp   ReplayPrep: the warp's share of the replay coefficients
-//              c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]} (d_j with q) and
-//              the self term k.q (RWKV6: r.(bonus*k)); then AppendDecode on
-//              its rows: read-out weights Gamma * k, Gamma * q (RWKV6:
-//              Gamma_{t-1} * r) formed per row, x = Sbar^T w partial sums,
-//              folded across the warp's row groups
-//   barrier 2  then the TV column threads finish x, replay the log on the
-//              value side, apply the delta correction and write the output
-// and a third before the stage is refilled.
-// Lambda_t = Lambda_{L-1} + g_t (RWKV6 reads at Lambda_{t-1}).
-// FOLD = false (append, "Fase di Append"): u_t, and (first tile of each
-//   head) k_t and Lambda_t, go to log slot L; the base is not written.
-// FOLD = true (merge-token, the token that completes the log: "Fase di
+// One CTA per unit (a head, or a TV-column value tile of a head).
+// ReplayPrep (once per CTA): decay point Lambda_t = Lambda_{L-1} + g_t
+// (RWKV6 reads at Lambda_{t-1}), read-out weights Gamma * k, Gamma * q (RWKV6:
+// Gamma * r), replay coefficients c_j = sum_i k_i k_j[i] e^{Lam[i] - Lam_j[i]}
+// (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
+// x = Sbar^T w over the register tile (the one base read), value-side replay,
+// delta correction, output.
+// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
+//   slot L; the base is not written.
+// FOLD = true (merge-token, the step that completes the log: "Fase di
 //   Merge"): the logical state after this token -- base decayed to Lambda_t,
 //   all L logged factors and this token's k u^T -- is written over the base
-//   tile (read once, written once); the caller resets the log (L = 0).
-template <int OP, int DK, int DV, int TV, int NT, int NS, bool FOLD>
+//   tile (the register tile is read once and written once); the log is left
+//   for the caller to reset (L = 0).
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
     static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
-    static_assert(NS >= 2 && NS <= 4, "pipeline depth");
 
     extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ float s_lt[DK];           // Lambda_t
+    __shared__ float s_lr[DK];           // decay point of read-out and replay
+    __shared__ float s_k[DK];
+    __shared__ float s_q[DK];
+    __shared__ float s_w[NA][DK];        // read-out weights
+    __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
+    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
-    __shared__ __align__(16) float s_red[T::NW][NA][TV];   // per-warp row partials
-    __shared__ float s_gam[FOLD ? DK : 1];
+    __shared__ __align__(16) float s_red[NA * T::NW * TV];
+    __shared__ float s_x[NA * TV];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int unit = blockIdx.x;
+    const int head = unit / T::NVT, vt = unit - head * T::NVT;
+    const int tid = threadIdx.x;
     const int L = p.L, C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
     const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
-    const int stage_bytes = up16(lay.bytes);
-    const int n_units = p.NH * T::NVT;
 
-    // fill one stage: small operands by warp 0, the tile by every thread
-    auto issue = [&](int unit, unsigned char *st) {
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        if (tid < 32) {
-            const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
-            stage_ops<OP, DK, DV, TV>(st, lay, src, head, vt, L, C, p.H, ie, true);
-        }
-        const float *bt = p.base + (size_t)head * DK * DV + vt * TV + c4;
-        unsigned char *tt = st + lay.tile + c4 * 4;
+    // 1. the base stream: RPT rows x 16 bytes per thread
+    float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
 #pragma unroll
-        for (int r = 0; r < T::RPT; ++r)
-            cp_async16(tt + (rg + r * T::RG) * TV * 4, bt + (size_t)(rg + r * T::RG) * DV);
-    };
+    for (int r = 0; r < T::RPT; ++r)
+        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
+                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
 
-#pragma unroll
-    for (int s = 0; s < NS - 1; ++s) {
-        const int u = blockIdx.x + s * gridDim.x;
-        if (u < n_units) issue(u, dsm + s * stage_bytes);
-        cp_async_commit();
+    // 2. small operands, staged by warp 0 while the base loads are in flight
+    if (tid < 32) {
+        const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true);
     }
+    __syncthreads();
+    const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
 
-    for (int it = 0;; ++it) {
-        const int unit = blockIdx.x + it * gridDim.x;
-        if (unit >= n_units) break;
-        {
-            const int un = unit + (NS - 1) * gridDim.x;
-            if (un < n_units) issue(un, dsm + ((it + NS - 1) % NS) * stage_bytes);
-            cp_async_commit();
+    // 3. key side: decay point, read-out weights (append: k_t, Lambda_t to slot L)
+    if (tid < DK) {
+        const int i = tid;
+        const int x = (OP == OP_GDN) ? 0 : i;
+        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+        const float lt = lprev + sg[x];
+        const float lr = (OP == OP_RWKV6) ? lprev : lt;
+        const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
+        const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
+        const float gam = expf(lr);
+        s_lt[i] = lt;
+        s_lr[i] = lr;
+        s_k[i] = kf;
+        s_q[i] = qf;
+        if (OP == OP_RWKV6) {
+            s_w[0][i] = gam * qf;
+            s_bk[i] = reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf;
+        } else {
+            s_w[0][i] = gam * kf;
+            s_w[NA - 1][i] = gam * qf;
         }
-        cp_async_wait_group<NS - 1>();
-        __syncthreads();                                    // barrier 1
-        unsigned char *st = dsm + (it % NS) * stage_bytes;
-        const int head = unit / T::NVT, vt = unit - head * T::NVT;
-        float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
-        unsigned char *tl = st + lay.tile + c4 * 4;
-
-        const float *sg = reinterpret_cast<const float *>(st + lay.g);
-        const float *slam = reinterpret_cast<const float *>(st + lay.lam);
-        const unsigned char *skin = st + lay.kin, *sqin = st + lay.qin;
-        // decay point of key channel i: Lambda_t (RWKV6: Lambda_{t-1})
-        auto lam_r = [&](int i) {
-            const int x = (OP == OP_GDN) ? 0 : i;
-            const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-            return (OP == OP_RWKV6) ? lprev : lprev + sg[x];
-        };
-
-        // 2a. key-side append of k_t and Lambda_t (first tile of the head)
-        if (!FOLD && vt == 0 && tid < DK) {
-            const int i = tid, x = (OP == OP_GDN) ? 0 : i;
-            const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, skin, i, p.in_bf16);
-            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lprev + sg[x];
+        if (!FOLD && vt == 0) {
+            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
+            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
         }
+    }
+    __syncthreads();
 
-        // 2b. ReplayPrep, this warp's share: task tau < L is log entry tau,
-        //     tau == L the self term
+    // replay coefficients: task tau < L is log entry tau, tau == L the self term
+    {
+        const int lane = tid & 31, warp = tid >> 5;
         for (int tau = warp; tau <= L; tau += T::NW) {
             float a0 = 0.f, a1 = 0.f;
             if (tau < L) {
-                const float gdec = (OP == OP_GDN) ? expf(lam_r(0) - slam[tau]) : 1.f;
+                const float gdec = (OP == OP_GDN) ? expf(s_lr[0] - slam[tau]) : 1.f;
 #pragma unroll
                 for (int i = lane; i < DK; i += 32) {
-                    const float kj = ld_raw(st + lay.K, tau * DK + i, p.in_bf16);
-                    const float e = (OP == OP_GDN) ? kj : expf(lam_r(i) - slam[tau * M + i]) * kj;
-                    const float qf = ld_raw(sqin, i, p.in_bf16);
+                    const float kj = ld_raw(dsm + lay.K, tau * DK + i, p.in_bf16);
+                    const float e = (OP == OP_GDN) ? kj : expf(s_lr[i] - slam[tau * M + i]) * kj;
                     if (OP == OP_RWKV6) {
-                        a0 = fmaf(qf, e, a0);
+                        a0 = fmaf(s_q[i], e, a0);
                     } else {
-                        a0 = fmaf(ld_raw(skin, i, p.in_bf16), e, a0);
-                        a1 = fmaf(qf, e, a1);
+                        a0 = fmaf(s_k[i], e, a0);
+                        a1 = fmaf(s_q[i], e, a1);
                     }
                 }
                 a0 = warp_sum(a0) * gdec;
@@ -475,138 +448,92 @@ append_kernel(const AppendParams p) {
                     if (NA == 2) s_coef[NA - 1][tau] = a1;
                 }
             } else {
-                const float *sbon = reinterpret_cast<const float *>(st + lay.bonus);
 #pragma unroll
-                for (int i = lane; i < DK; i += 32) {
-                    const float kf = ld_raw(skin, i, p.in_bf16), qf = ld_raw(sqin, i, p.in_bf16);
-                    a0 = fmaf(qf, (OP == OP_RWKV6) ? sbon[i] * kf : kf, a0);
-                }
+                for (int i = lane; i < DK; i += 32)
+                    a0 = fmaf(s_q[i], (OP == OP_RWKV6) ? s_bk[i] : s_k[i], a0);
                 a0 = warp_sum(a0);
                 if (lane == 0) s_self = a0;
             }
         }
-
-        // 2c. AppendDecode on this thread's rows of the staged tile:
-        //     x_a[c] = sum_i w_a[i] * Sbar[i][c], weights formed per row
-        {
-            const float gsc = (OP == OP_GDN) ? expf(lam_r(0)) : 1.f;
-            float4 acc[NA];
-#pragma unroll
-            for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const int row = rg + r * T::RG;
-                const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
-                const float gam = (OP == OP_GDN) ? gsc : expf(lam_r(row));
-                float w[NA];
-                if (OP == OP_RWKV6) {
-                    w[0] = gam * ld_raw(sqin, row, p.in_bf16);
-                } else {
-                    w[0] = gam * ld_raw(skin, row, p.in_bf16);
-                    w[NA - 1] = gam * ld_raw(sqin, row, p.in_bf16);
-                }
-#pragma unroll
-                for (int a = 0; a < NA; ++a) {
-                    acc[a].x = fmaf(w[a], sv.x, acc[a].x);
-                    acc[a].y = fmaf(w[a], sv.y, acc[a].y);
-                    acc[a].z = fmaf(w[a], sv.z, acc[a].z);
-                    acc[a].w = fmaf(w[a], sv.w, acc[a].w);
-                }
-            }
-            // fold the warp's row groups, then one row of partials per warp
-#pragma unroll
-            for (int a = 0; a < NA; ++a) {
-#pragma unroll
-                for (int o = T::TPR; o < 32; o <<= 1) {
-                    acc[a].x += __shfl_xor_sync(0xffffffffu, acc[a].x, o);
-                    acc[a].y += __shfl_xor_sync(0xffffffffu, acc[a].y, o);
-                    acc[a].z += __shfl_xor_sync(0xffffffffu, acc[a].z, o);
-                    acc[a].w += __shfl_xor_sync(0xffffffffu, acc[a].w, o);
-                }
-                if (lane < T::TPR) *reinterpret_cast<float4 *>(&s_red[warp][a][c4]) = acc[a];
-            }
-        }
-        __syncthreads();                                        // barrier 2
-
-        // 3. value side: finish x, log replay, delta correction, output, append of u
-        if (tid < TV) {
-            const int c = tid;
-            const int col = vt * TV + c;
-            const size_t ub = (size_t)head * C * DV + col;
-            float x[NA];
-#pragma unroll
-            for (int a = 0; a < NA; ++a) {
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < T::NW; ++w) sum += s_red[w][a][c];
-                x[a] = sum;
-            }
-            const float vv = ld_raw(st + lay.vin, c, p.in_bf16);
-            if (OP == OP_RWKV6) {
-                float rr = 0.f;
-                for (int j = 0; j < L; ++j) rr = fmaf(s_coef[0][j], ld_raw(st + lay.U, j * TV + c, p.in_bf16), rr);
-                const float o = p.scale * (x[0] + rr + s_self * vv);
-                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-                if (FOLD)
-                    s_u[c] = vv;
-                else
-                    copy_raw(p.logU, ub + (size_t)L * DV, st + lay.vin, c, p.in_bf16);
-            } else {
-                const float *U = reinterpret_cast<const float *>(st + lay.U);
-                float rk = 0.f, rq = 0.f;
-                for (int j = 0; j < L; ++j) {
-                    const float uj = U[j * TV + c];
-                    rk = fmaf(s_coef[0][j], uj, rk);
-                    rq = fmaf(s_coef[1][j], uj, rq);
-                }
-                const float beta = *reinterpret_cast<const float *>(st + lay.beta);
-                const float u = beta * (vv - x[0] - rk);
-                const float o = p.scale * (x[NA - 1] + rq + s_self * u);
-                st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-                if (FOLD)
-                    s_u[c] = u;
-                else
-                    reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
-            }
-        }
-
-        // 4. merge-token: write the logical state after this token over the base
-        if (FOLD) {
-            // replay-factor table with Lambda_t, then the new rows
-            float *A = reinterpret_cast<float *>(st + lay.A);
-            {
-                const int AP = up4(L) + 4;
-                for (int idx = tid; idx < DK * (L + 1); idx += NT) {
-                    const int i = idx % DK, j = idx / DK;
-                    const int x = (OP == OP_GDN) ? 0 : i;
-                    const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
-                    const float lt = lprev + sg[x];
-                    if (j == L)
-                        s_gam[i] = expf(lt);
-                    else
-                        A[i * AP + j] = expf(lt - slam[j * M + x]) * ld_raw(st + lay.K, j * DK + i, p.in_bf16);
-                }
-            }
-            __syncthreads();
-            const int AP = up4(L) + 4;
-            const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-            const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const int row = rg + r * T::RG;
-                const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
-                float4 o = fold_row<TV>(sv, s_gam[row], A + row * AP, st + lay.U, c4, L, ubf);
-                const float kr = ld_raw(skin, row, p.in_bf16);
-                o.x = fmaf(kr, u4.x, o.x);
-                o.y = fmaf(kr, u4.y, o.y);
-                o.z = fmaf(kr, u4.z, o.z);
-                o.w = fmaf(kr, u4.w, o.w);
-                st_state(bh + (size_t)row * DV, o);
-            }
-        }
-        __syncthreads();   // the stage and the shared partials are reused next
     }
-    cp_async_wait_group<0>();
+    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
+                                       dsm + lay.K, slam, L, p.in_bf16);
+    __syncthreads();
+
+    // 4. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    {
+        float4 acc[NA];
+#pragma unroll
+        for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+#pragma unroll
+            for (int a = 0; a < NA; ++a) {
+                const float w = s_w[a][row];
+                acc[a].x = fmaf(w, s[r].x, acc[a].x);
+                acc[a].y = fmaf(w, s[r].y, acc[a].y);
+                acc[a].z = fmaf(w, s[r].z, acc[a].z);
+                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+            }
+        }
+        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
+    }
+
+    // 5. value side: log replay, delta correction, output, append of u
+    if (tid < TV) {
+        const int c = tid;
+        const int col = vt * TV + c;
+        const size_t ub = (size_t)head * C * DV + col;
+        const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
+        if (OP == OP_RWKV6) {
+            float rr = 0.f;
+            for (int j = 0; j < L; ++j)
+                rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
+            const float o = p.scale * (s_x[c] + rr + s_self * vv);
+            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+            if (FOLD)
+                s_u[c] = vv;
+            else
+                copy_raw(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16);
+        } else {
+            const float *U = reinterpret_cast<const float *>(dsm + lay.U);
+            float rk = 0.f, rq = 0.f;
+            for (int j = 0; j < L; ++j) {
+                const float uj = U[j * TV + c];
+                rk = fmaf(s_coef[0][j], uj, rk);
+                rq = fmaf(s_coef[1][j], uj, rq);
+            }
+            const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
+            const float u = beta * (vv - s_x[c] - rk);
+            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+            st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
+            if (FOLD)
+                s_u[c] = u;
+            else
+                reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
+        }
+    }
+
+    // 6. merge-token: write the logical state after this token over the base
+    if (FOLD) {
+        __syncthreads();
+        const float *A = reinterpret_cast<const float *>(dsm + lay.A);
+        const int AP = up4(L) + 4;
+        const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+        const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+            const float kr = s_k[row];
+            o.x = fmaf(kr, u4.x, o.x);
+            o.y = fmaf(kr, u4.y, o.y);
+            o.z = fmaf(kr, u4.z, o.z);
+            o.w = fmaf(kr, u4.w, o.w);
+            st_state(bh + (size_t)row * DV, o);
+        }
+    }
 }
 
 // ================================================= merge / materialise ==
@@ -637,17 +564,14 @@ merge_kernel(const MergeParams p) {
 
     const float *bh = p.base + (size_t)head * DK * DV + vt * TV + c4;
     float *dh = p.dst + (size_t)head * DK * DV + vt * TV + c4;
+    float4 s[T::RPT];
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
+
     if (tid < 32) {
         const OpSources src{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
         stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false);
     }
-    cp_async_commit();
-    unsigned char *tl = dsm + lay.tile + c4 * 4;
-#pragma unroll
-    for (int r = 0; r < T::RPT; ++r)
-        cp_async16(tl + (rg + r * T::RG) * TV * 4, bh + (size_t)(rg + r * T::RG) * DV);
-    cp_async_commit();
-    cp_async_wait_group<1>();
     __syncthreads();
     const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
     for (int x = tid; x < M; x += NT) s_lL[x] = L > 0 ? slam[(L - 1) * M + x] : 0.f;
@@ -659,12 +583,10 @@ merge_kernel(const MergeParams p) {
     const float *A = reinterpret_cast<const float *>(dsm + lay.A);
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-    cp_async_wait_group<0>();
 #pragma unroll
     for (int r = 0; r < T::RPT; ++r) {
         const int row = rg + r * T::RG;
-        const float4 sv = *reinterpret_cast<const float4 *>(tl + row * TV * 4);
-        st_state(dh + (size_t)row * DV, fold_row<TV>(sv, s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
     }
 }
 

@@ -4,7 +4,6 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "kernels.cuh"
 
@@ -25,59 +24,14 @@ cudaError_t sm_count(int *sms);
 
 // Value-tile width for NH heads of width DV: 64 columns (or the whole head
 // when narrower) while that still gives at least four CTAs per SM, else the
-// widest tile that does (>= 32 columns).
+// widest tile that does (>= 32 columns).  Measured on B200 for d = 64 and 128:
+// 64-column tiles beat 32 (more per-CTA work to amortise the prologue) and
+// 128 (fewer, longer CTAs: worse overlap of their serial phases).
 inline int pick_tile(long long NH, int DV, int sms) {
     int tv = DV < 64 ? DV : 64;
     while (tv > 32 && NH * (DV / tv) < 4LL * sms) tv /= 2;
     return tv;
 }
-
-// Pipeline depth (stages) of the persistent append kernel per tile width.
-template <int TV>
-struct Pipe {
-    static constexpr int NS = (TV == 32) ? 3 : 2;
-};
-
-// Resident CTAs per SM of a kernel at a given dynamic shared-memory size,
-// cached per (device, size).
-class OccupancyCache {
-   public:
-    template <typename Kernel>
-    cudaError_t get(Kernel kern, int nt, size_t smem, int *per_sm) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        {
-            std::lock_guard<std::mutex> lock(mu_);
-            for (int i = 0; i < n_; ++i)
-                if (dev_[i] == dev && smem_[i] == smem) {
-                    *per_sm = occ_[i];
-                    return cudaSuccess;
-                }
-        }
-        int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nt, smem);
-        if (e != cudaSuccess) return e;
-        if (occ < 1) return cudaErrorInvalidConfiguration;
-        std::lock_guard<std::mutex> lock(mu_);
-        if (n_ < kSlots) {
-            dev_[n_] = dev;
-            smem_[n_] = smem;
-            occ_[n_] = occ;
-            ++n_;
-        }
-        *per_sm = occ;
-        return cudaSuccess;
-    }
-
-   private:
-    static constexpr int kSlots = 64;
-    std::mutex mu_;
-    int dev_[kSlots] = {};
-    size_t smem_[kSlots] = {};
-    int occ_[kSlots] = {};
-    int n_ = 0;
-};
 
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename Kernel>
