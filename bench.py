@@ -220,41 +220,43 @@ def recorded_traffic(workload_name):
 # ------------------------------------------------------- CPU oracle -----
 
 def cpu_oracle_sample(w, target_s=12.0, seed=99):
-    """Time the fp64 oracle's base+log decode on a bounded sample of heads
-    of the workload (one merge cycle of C tokens); returns tok/s in the
-    GPU's unit (head-tokens per second / H), the threads used and a note."""
+    """Time the fp64 oracle's base+log decode on a bounded sample of the
+    workload -- a random subset of its heads over whole merge cycles -- sized
+    to about `target_s` seconds of host work.  Returns tok/s in the GPU's
+    unit (head-tokens per second / H), the threads used and the sample."""
     import oracle
     from recurrent_state_head_b200 import synth
 
     threads = max(1, len(os.sched_getaffinity(0)))
     rng = np.random.default_rng(seed)
+    S_all = synth.initial_state(w).reshape(w.heads, w.dk, w.dv)
+    bon_all = synth.bonus(w)
 
-    def run(n_heads):
+    def run(n_heads, n_cycles):
         heads = np.sort(rng.choice(w.heads, size=min(n_heads, w.heads), replace=False))
-        ti = synth.tokens(w, 0, w.C, heads=heads)
-        S0 = synth.initial_state(w).reshape(w.heads, w.dk, w.dv)[heads]
-        bon = synth.bonus(w)
-        bon = None if bon is None else bon[heads % w.H]
+        T = n_cycles * w.C
+        ti = synth.tokens(w, 0, T, heads=heads)
         g = ti.g.astype(np.float64)
         if g.ndim == 2:
             g = g[:, :, None]
-        st = oracle.LogState(w.op, S0, w.C)
+        bon = None if bon_all is None else bon_all[heads % w.H]
+        st = oracle.LogState(w.op, S_all[heads], w.C)
         t0 = time.perf_counter()
         oracle.deltalog_run(st, ti.q64, ti.k64, ti.v64,
                             None if w.op == 2 else ti.beta.astype(np.float64), g, bon,
                             w.scale, n_threads=threads)
-        return time.perf_counter() - t0, len(heads)
+        return time.perf_counter() - t0, len(heads), T
 
-    probe_heads = max(threads, 8)
-    dt, n = run(probe_heads)
-    per_head = dt / n
-    n_heads = int(max(probe_heads, min(w.heads, target_s / max(per_head, 1e-9))))
-    dt, n = run(n_heads)
-    head_tokens = n * w.C
-    return {"value": head_tokens / dt / w.H, "unit": "tok/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"{n} of {w.heads} heads x {w.C} tokens (one merge cycle), "
-                      f"fp64 base+log oracle, {dt:.1f} s"}
+    probe = min(w.heads, max(4 * threads, 16))
+    dt, n, T = run(probe, 1)
+    per_head_token = dt / (n * T)
+    budget = target_s / max(per_head_token, 1e-9)            # head-tokens to run
+    n_heads = int(min(w.heads, max(probe, budget / w.C)))
+    n_cycles = int(max(1, min(w.T // w.C, budget / (n_heads * w.C))))
+    dt, n, T = run(n_heads, n_cycles)
+    return {"value": n * T / dt / w.H, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {w.heads} heads x {T} tokens ({n_cycles} merge cycles), "
+                      f"fp64 base+log oracle, {dt:.1f} s on {threads} threads"}
 
 
 # ------------------------------------------------------------ native ----
