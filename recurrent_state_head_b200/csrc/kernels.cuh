@@ -133,6 +133,23 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// acc += w * s on four lanes as two paired fp32 FMAs (sm_100 FFMA2; each
+// lane is one correctly rounded fused multiply-add, as fmaf)
+__device__ __forceinline__ void fma4(float4 &acc, float w, const float4 &s) {
+    const float2 ww = make_float2(w, w);
+    const float2 lo = __ffma2_rn(ww, make_float2(s.x, s.y), make_float2(acc.x, acc.y));
+    const float2 hi = __ffma2_rn(ww, make_float2(s.z, s.w), make_float2(acc.z, acc.w));
+    acc = make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// a * s + b * t on four lanes
+__device__ __forceinline__ float4 fma4_2(float a, const float4 &s, float b, const float4 &t) {
+    const float2 aa = make_float2(a, a), bb = make_float2(b, b);
+    const float2 lo = __ffma2_rn(aa, make_float2(s.x, s.y), __fmul2_rn(bb, make_float2(t.x, t.y)));
+    const float2 hi = __ffma2_rn(aa, make_float2(s.z, s.w), __fmul2_rn(bb, make_float2(t.z, t.w)));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -313,18 +330,16 @@ __device__ __forceinline__ void replay_table(float *A, float *gam, const float *
 template <int TV>
 __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow, const unsigned char *sU,
                                            int c4, int L, int ubf) {
-    float4 o = make_float4(gm * s.x, gm * s.y, gm * s.z, gm * s.w);
+    const float2 g2 = make_float2(gm, gm);
+    const float2 olo = __fmul2_rn(g2, make_float2(s.x, s.y)), ohi = __fmul2_rn(g2, make_float2(s.z, s.w));
+    float4 o = make_float4(olo.x, olo.y, ohi.x, ohi.y);
     for (int j0 = 0; j0 < L; j0 += 4) {
         const float4 cf4 = *reinterpret_cast<const float4 *>(Arow + j0);
         const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             if (j0 + jj < L) {
-                const float4 u = ld_raw4(sU, (j0 + jj) * TV + c4, ubf);
-                o.x = fmaf(cf[jj], u.x, o.x);
-                o.y = fmaf(cf[jj], u.y, o.y);
-                o.z = fmaf(cf[jj], u.z, o.z);
-                o.w = fmaf(cf[jj], u.w, o.w);
+                fma4(o, cf[jj], ld_raw4(sU, (j0 + jj) * TV + c4, ubf));
             }
         }
     }
@@ -471,10 +486,7 @@ append_kernel(const AppendParams p) {
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
                 const float w = s_w[a][row];
-                acc[a].x = fmaf(w, s[r].x, acc[a].x);
-                acc[a].y = fmaf(w, s[r].y, acc[a].y);
-                acc[a].z = fmaf(w, s[r].z, acc[a].z);
-                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+                fma4(acc[a], w, s[r]);
             }
         }
         reduce_rows<NA, TV, NT>(acc, s_red, s_x);
@@ -526,11 +538,7 @@ append_kernel(const AppendParams p) {
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
             float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-            const float kr = s_k[row];
-            o.x = fmaf(kr, u4.x, o.x);
-            o.y = fmaf(kr, u4.y, o.y);
-            o.z = fmaf(kr, u4.z, o.z);
-            o.w = fmaf(kr, u4.w, o.w);
+            fma4(o, s_k[row], u4);
             st_state(bh + (size_t)row * DV, o);
         }
     }
@@ -664,13 +672,8 @@ eager_kernel(const EagerParams p) {
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
             const float w = s_w[0][row], a = s_a[row], kr = s_k[row];
-            acc[0].x = fmaf(w, s[r].x, acc[0].x);
-            acc[0].y = fmaf(w, s[r].y, acc[0].y);
-            acc[0].z = fmaf(w, s[r].z, acc[0].z);
-            acc[0].w = fmaf(w, s[r].w, acc[0].w);
-            st_state(Sh + (size_t)row * DV + col0,
-                     make_float4(fmaf(a, s[r].x, kr * v4.x), fmaf(a, s[r].y, kr * v4.y),
-                                 fmaf(a, s[r].z, kr * v4.z), fmaf(a, s[r].w, kr * v4.w)));
+            fma4(acc[0], w, s[r]);
+            st_state(Sh + (size_t)row * DV + col0, fma4_2(a, s[r], kr, v4));
         }
         reduce_rows<NA, TV, NT>(acc, s_red, s_x);
         for (int c = tid; c < TV; c += NT) {
@@ -685,10 +688,7 @@ eager_kernel(const EagerParams p) {
 #pragma unroll
             for (int a = 0; a < NA; ++a) {
                 const float w = s_w[a][row];
-                acc[a].x = fmaf(w, s[r].x, acc[a].x);
-                acc[a].y = fmaf(w, s[r].y, acc[a].y);
-                acc[a].z = fmaf(w, s[r].z, acc[a].z);
-                acc[a].w = fmaf(w, s[r].w, acc[a].w);
+                fma4(acc[a], w, s[r]);
             }
         }
         reduce_rows<NA, TV, NT>(acc, s_red, s_x);
@@ -705,9 +705,7 @@ eager_kernel(const EagerParams p) {
         for (int r = 0; r < T::RPT; ++r) {
             const int row = rg + r * T::RG;
             const float a = s_a[row], kr = s_k[row];
-            st_state(Sh + (size_t)row * DV + col0,
-                     make_float4(fmaf(a, s[r].x, kr * u4.x), fmaf(a, s[r].y, kr * u4.y),
-                                 fmaf(a, s[r].z, kr * u4.z), fmaf(a, s[r].w, kr * u4.w)));
+            st_state(Sh + (size_t)row * DV + col0, fma4_2(a, s[r], kr, u4));
         }
     }
 }
