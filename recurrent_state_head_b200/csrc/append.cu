@@ -8,7 +8,7 @@ namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
-    constexpr int NT = 4 * TV;
+    constexpr int NT = CtaShape<DK, TV>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD>;
     const int ie = p.in_bf16 ? 2 : 4;

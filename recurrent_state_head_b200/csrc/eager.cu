@@ -6,7 +6,7 @@ namespace {
 template <int OP, int DK, int DV>
 cudaError_t launch(const EagerParams &p, cudaStream_t s) {
     // one CTA per (head, 32-column tile), tile held in registers
-    constexpr int TV = 32, NT = 128;
+    constexpr int TV = 32, NT = CtaShape<DK, TV>::NT;
     const unsigned grid = (unsigned)p.NH * (DV / TV);
     eager_kernel<OP, DK, DV, TV, NT><<<grid, NT, 0, s>>>(p);
     return cudaGetLastError();

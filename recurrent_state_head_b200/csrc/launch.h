@@ -33,6 +33,14 @@ inline int pick_tile(long long NH, int DV, int sms) {
     return tv;
 }
 
+// Threads of a CTA over a TV-column tile of d_k rows: TV/4 threads per row
+// (one 16-byte column group each) and d_k/8 row groups, so that every thread
+// streams 8 rows of its column group.
+template <int DK, int TV>
+struct CtaShape {
+    static constexpr int NT = (TV / 4) * (DK / 8);
+};
+
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename Kernel>
 cudaError_t allow_smem(std::atomic<unsigned long long> &done, Kernel kern, size_t bytes) {

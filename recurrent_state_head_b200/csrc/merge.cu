@@ -5,7 +5,7 @@ namespace dl {
 namespace {
 template <int OP, int DK, int DV, int TV>
 cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
-    constexpr int NT = 4 * TV;
+    constexpr int NT = CtaShape<DK, TV>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = merge_kernel<OP, DK, DV, TV, NT>;
     const int ie = p.in_bf16 ? 2 : 4;
