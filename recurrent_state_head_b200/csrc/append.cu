@@ -16,8 +16,23 @@ cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)p.NH * (DV / TV);
-    kern<<<grid, NT, smem, s>>>(p);
-    return cudaGetLastError();
+    if (!p.early) {
+        kern<<<grid, NT, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    // programmatic dependent launch: may start while the previous kernel of
+    // the stream finishes (the kernel orders itself with griddepcontrol)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <int OP, int DK, int DV, bool FOLD>

@@ -134,6 +134,7 @@ dl::AppendParams append_params(const dl_handle *h, const dl_step_io &io, int L) 
     p.scale = h->cfg.scale;
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
     p.out_bf16 = h->cfg.out_dtype == DL_BF16;
+    p.early = 0;
     return p;
 }
 
@@ -153,9 +154,29 @@ dl::MergeParams merge_params(const dl_handle *h, float *dst, int L) {
 
 // fold: the merge-token variant (the token that completes the log writes
 // the merged state over the base instead of appending).
-cudaError_t launch_append(const dl_handle *h, const dl_step_io &io, int L, bool fold, cudaStream_t s) {
+// early: launch as a programmatic dependent that streams its base before the
+// previous kernel of the stream has finished -- only where that kernel cannot
+// be writing this base (a merge cycle over several layers with distinct
+// bases).
+cudaError_t launch_append(const dl_handle *h, const dl_step_io &io, int L, bool fold, cudaStream_t s,
+                          bool early = false) {
     if (h->NH == 0) return cudaSuccess;
-    return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(append_params(h, io, L), fold, s);
+    dl::AppendParams p = append_params(h, io, L);
+    p.early = early ? 1 : 0;
+    return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, fold, s);
+}
+
+// Do the layers' base states occupy pairwise disjoint memory?
+bool disjoint_bases(dl_handle *const *layers, int n) {
+    for (int a = 0; a < n; ++a)
+        for (int b = a + 1; b < n; ++b) {
+            const char *pa = reinterpret_cast<const char *>(layers[a]->base);
+            const char *pb = reinterpret_cast<const char *>(layers[b]->base);
+            const size_t na = (size_t)layers[a]->NH * layers[a]->cfg.dk * layers[a]->cfg.dv * 4;
+            const size_t nb = (size_t)layers[b]->NH * layers[b]->cfg.dk * layers[b]->cfg.dv * 4;
+            if (na && nb && pa < pb + nb && pb < pa + na) return false;
+        }
+    return true;
 }
 
 cudaError_t launch_merge(const dl_handle *h, float *dst, int L, cudaStream_t s) {
@@ -326,6 +347,10 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
         delete cy;
         return fail(DL_ENOMEM, "host allocation of the cycle failed");
     }
+    // with two or more layers on disjoint bases, consecutive kernels of the
+    // token-major cycle belong to different layers: each may start streaming
+    // its base during the previous kernel's tail
+    const bool overlap = n_layers >= 2 && disjoint_bases(layers, n_layers);
     cudaStream_t st = nullptr;
     cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
     if (e != cudaSuccess) {
@@ -343,7 +368,7 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
                 const dl_handle *h = layers[l];
                 const bool last = t == C - 1;
                 const bool fold = last && h->cfg.auto_merge == DL_MERGE_FOLD;
-                le = launch_append(h, io[(size_t)t * n_layers + l], t, fold, st);
+                le = launch_append(h, io[(size_t)t * n_layers + l], t, fold, st, overlap);
                 if (h->NH > 0) cy->kernels += 1;
                 if (le == cudaSuccess && last && h->cfg.auto_merge == DL_MERGE_SEPARATE) {
                     le = launch_merge(h, h->base, C, st);

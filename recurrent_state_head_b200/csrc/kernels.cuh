@@ -41,6 +41,10 @@ struct AppendParams {
     int NH, H, C, L;
     float scale;
     int in_bf16, out_bf16;
+    int early;                // 1: stream the base before waiting for the
+                              // previous kernel (launch is a programmatic
+                              // dependent and the previous kernel does not
+                              // write this base)
 };
 
 struct MergeParams {
@@ -393,13 +397,23 @@ append_kernel(const AppendParams p) {
     const int c4 = col4 * 4;
     const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
 
-    // 1. the base stream: RPT rows x 16 bytes per thread
+    // 1. the base stream: RPT rows x 16 bytes per thread.  As a programmatic
+    //    dependent launch (merge cycles over several layers) the stream
+    //    starts before the previous kernel -- another layer's -- has
+    //    finished; everything else this kernel reads or writes comes after
+    //    griddepcontrol.wait (a no-op for an ordinary launch).
     float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
     float4 s[T::RPT];
+    auto load_base = [&]() {
 #pragma unroll
-    for (int r = 0; r < T::RPT; ++r)
-        s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
-                    : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+        for (int r = 0; r < T::RPT; ++r)
+            s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
+                        : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+    };
+    if (p.early) load_base();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!p.early) load_base();
 
     // 2. small operands, staged by warp 0 while the base loads are in flight
     if (tid < 32) {
