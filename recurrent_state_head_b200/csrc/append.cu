@@ -6,11 +6,11 @@
 
 namespace dl {
 namespace {
-template <int OP, int DK, int DV, int TV, bool FOLD>
-cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
+template <int OP, int DK, int DV, int TV, bool FOLD, int LB>
+cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = CtaShape<DK, TV>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD>;
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
@@ -33,6 +33,17 @@ cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// The merge-token keeps the logged value factors in registers while the log
+// is short (L <= 3 or L <= 7); longer logs are read from shared memory.
+template <int OP, int DK, int DV, int TV, bool FOLD>
+cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
+    if constexpr (FOLD) {
+        if (p.L <= 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
+        if (p.L <= 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
+    }
+    return launch_lb<OP, DK, DV, TV, FOLD, 0>(p, s);
 }
 
 template <int OP, int DK, int DV, bool FOLD>

@@ -350,6 +350,27 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
     return o;
 }
 
+// The same with the L <= LB value factors of this thread's four columns held
+// in registers (loaded once, reused for every row of the tile).
+template <int LB>
+__device__ __forceinline__ float4 fold_row_reg(float4 s, float gm, const float *Arow,
+                                               const float4 (&ur)[LB], int L) {
+    const float2 g2 = make_float2(gm, gm);
+    const float2 olo = __fmul2_rn(g2, make_float2(s.x, s.y)), ohi = __fmul2_rn(g2, make_float2(s.z, s.w));
+    float4 o = make_float4(olo.x, olo.y, ohi.x, ohi.y);
+#pragma unroll
+    for (int j0 = 0; j0 < LB; j0 += 4) {
+        if (j0 < L) {
+            const float4 cf4 = *reinterpret_cast<const float4 *>(Arow + j0);
+            const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                if (j0 + jj < LB && j0 + jj < L) fma4(o, cf[jj], ur[j0 + jj]);
+        }
+    }
+    return o;
+}
+
 // ============================================ append + read-out (+ fold) ==
 //
 // One CTA per unit (a head, or a TV-column value tile of a head).
@@ -366,7 +387,7 @@ __device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow
 //   all L logged factors and this token's k u^T -- is written over the base
 //   tile (the register tile is read once and written once); the log is left
 //   for the caller to reset (L = 0).
-template <int OP, int DK, int DV, int TV, int NT, bool FOLD>
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0>
 __global__ void __launch_bounds__(NT)
 append_kernel(const AppendParams p) {
     using T = Tile<DK, DV, TV, NT>;
@@ -548,12 +569,27 @@ append_kernel(const AppendParams p) {
         const int AP = up4(L) + 4;
         const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
         const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
+        if constexpr (LB > 0) {
+            // the logged value factors of this thread's columns, once
+            float4 ur[LB];
 #pragma unroll
-        for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-            fma4(o, s_k[row], u4);
-            st_state(bh + (size_t)row * DV, o);
+            for (int j = 0; j < LB; ++j)
+                ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < T::RPT; ++r) {
+                const int row = rg + r * T::RG;
+                float4 o = fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L);
+                fma4(o, s_k[row], u4);
+                st_state(bh + (size_t)row * DV, o);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < T::RPT; ++r) {
+                const int row = rg + r * T::RG;
+                float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+                fma4(o, s_k[row], u4);
+                st_state(bh + (size_t)row * DV, o);
+            }
         }
     }
 }
