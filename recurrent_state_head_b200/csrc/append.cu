@@ -36,12 +36,12 @@ cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
 }
 
 // The merge-token keeps the logged value factors in registers while the log
-// is short (L <= 3 or L <= 7); longer logs are read from shared memory.
+// is short (up to 8 entries); longer logs are read from shared memory.
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     if constexpr (FOLD) {
-        if (p.L <= 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
-        if (p.L <= 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
+        if (p.L <= 4) return launch_lb<OP, DK, DV, TV, true, 4>(p, s);
+        if (p.L <= 8) return launch_lb<OP, DK, DV, TV, true, 8>(p, s);
     }
     return launch_lb<OP, DK, DV, TV, FOLD, 0>(p, s);
 }

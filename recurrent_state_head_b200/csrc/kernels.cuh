@@ -601,7 +601,7 @@ append_kernel(const AppendParams p) {
 // (dst == base) it is the merge; into another buffer it is materialise.
 // One CTA per unit; the register tile is loaded first, the log staged by
 // warp 0, the replay-factor table built once per CTA.
-template <int OP, int DK, int DV, int TV, int NT>
+template <int OP, int DK, int DV, int TV, int NT, int LB = 0>
 __global__ void __launch_bounds__(NT)
 merge_kernel(const MergeParams p) {
     using T = Tile<DK, DV, TV, NT>;
@@ -641,10 +641,24 @@ merge_kernel(const MergeParams p) {
     const float *A = reinterpret_cast<const float *>(dsm + lay.A);
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+    if constexpr (LB > 0) {
+        // the logged value factors of this thread's columns, once
+        float4 ur[LB];
 #pragma unroll
-    for (int r = 0; r < T::RPT; ++r) {
-        const int row = rg + r * T::RG;
-        st_state(dh + (size_t)row * DV, fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        for (int j = 0; j < LB; ++j)
+            ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            st_state(dh + (size_t)row * DV, fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L));
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            st_state(dh + (size_t)row * DV,
+                     fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+        }
     }
 }
 

@@ -3,11 +3,11 @@
 
 namespace dl {
 namespace {
-template <int OP, int DK, int DV, int TV>
-cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
+template <int OP, int DK, int DV, int TV, int LB>
+cudaError_t launch_lb(const MergeParams &p, cudaStream_t s) {
     constexpr int NT = CtaShape<DK, TV>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = merge_kernel<OP, DK, DV, TV, NT>;
+    auto kern = merge_kernel<OP, DK, DV, TV, NT, LB>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, true).bytes;
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, true).bytes);
@@ -15,6 +15,14 @@ cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
     const unsigned grid = (unsigned)p.NH * (DV / TV);
     kern<<<grid, NT, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+// The logged value factors stay in registers for logs of up to 8 entries.
+template <int OP, int DK, int DV, int TV>
+cudaError_t launch_tv(const MergeParams &p, cudaStream_t s) {
+    if (p.L <= 4) return launch_lb<OP, DK, DV, TV, 4>(p, s);
+    if (p.L <= 8) return launch_lb<OP, DK, DV, TV, 8>(p, s);
+    return launch_lb<OP, DK, DV, TV, 0>(p, s);
 }
 
 template <int OP, int DK, int DV>
