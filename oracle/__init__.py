@@ -6,5 +6,5 @@ with, or called by, the CUDA path.
 """
 from .oracle import (  # noqa: F401
     GDN, KDA, RWKV6, OP_NAMES, LogState, build, decay_width, eager_run,
-    deltalog_run, materialize, merge, max_threads, rel_err,
+    deltalog_run, deltalog_slots_run, materialize, merge, max_threads, rel_err,
 )

@@ -283,6 +283,66 @@ int oracle_deltalog_run(int op, int nh, int dk, int dv, int C, int T, double sca
     return 0;
 }
 
+/* Base+log decode with a log length per slot (continuous batching: slots
+ * join, leave and idle independently, so their logs fill at different
+ * tokens).  Heads are grouped by slot, head = s * H + h for slot s < nslots.
+ * Slot s takes part in token t only when active[t * nslots + s] is nonzero:
+ * then each of its heads appends at the slot's own log length, and the slot
+ * merges when its log is full; an idle slot's heads, log and output rows are
+ * left untouched.  Ls[s] is slot s's log length on entry and on exit;
+ * L_trace[t * nslots + s] = slot s's length after token t (may be NULL).
+ * Returns 0, or 1 on bad arguments. */
+int oracle_deltalog_slots_run(int op, int nslots, int H, int dk, int dv, int C, int T,
+                              double scale, double *base, double *K, double *U, double *Lam,
+                              int *Ls, const unsigned char *active,
+                              const double *q, const double *k, const double *v,
+                              const double *beta, const double *g, const double *bonus,
+                              double *out, int *L_trace, int n_threads)
+{
+    if (op < 0 || op > 2 || nslots < 0 || H < 1 || dk <= 0 || dv <= 0 || T < 0) return 1;
+    if (C < 1 || C > 64 || dk > 1024 || dv > 1024) return 1;
+    for (int s = 0; s < nslots; ++s)
+        if (Ls[s] < 0 || Ls[s] >= C) return 1;
+    const int m = decay_width(op, dk);
+    const int nh = nslots * H;
+    if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for num_threads(n_threads) schedule(dynamic, 1)
+    for (int hh = 0; hh < nh; ++hh) {
+        const int s = hh / H;
+        double *bh = base + (size_t)hh * dk * dv;
+        double *Kh = K + (size_t)hh * C * dk;
+        double *Uh = U + (size_t)hh * C * dv;
+        double *Lh = Lam + (size_t)hh * C * m;
+        int L = Ls[s];
+        for (int t = 0; t < T; ++t) {
+            if (!active[(size_t)t * nslots + s]) continue;
+            size_t th = (size_t)t * nh + hh;
+            append_step_head(op, dk, dv, C, scale, bh, Kh, Uh, Lh, L,
+                             q + th * dk, k + th * dk, v + th * dv,
+                             beta ? beta[th] : 0.0, g + th * m,
+                             bonus ? bonus + (size_t)hh * dk : NULL, out + th * dv);
+            L += 1;
+            if (L == C) {
+                materialize_head(op, dk, dv, bh, Kh, Uh, Lh, L, bh);
+                L = 0;
+            }
+        }
+    }
+    /* the per-slot schedule depends only on the activity pattern */
+    for (int s = 0; s < nslots; ++s) {
+        int L = Ls[s];
+        for (int t = 0; t < T; ++t) {
+            if (active[(size_t)t * nslots + s]) {
+                L += 1;
+                if (L == C) L = 0;
+            }
+            if (L_trace) L_trace[(size_t)t * nslots + s] = L;
+        }
+        Ls[s] = L;
+    }
+    return 0;
+}
+
 /* Out-of-place materialisation of nh heads with log length L. */
 int oracle_materialize(int op, int nh, int dk, int dv, int C, int L,
                        const double *base, const double *K, const double *U,

@@ -53,10 +53,12 @@ def _load():
             lib.oracle_eager_run.argtypes = [i, i, i, i, i, d, P, P, P, P, P, P, P, P, P, i]
             lib.oracle_deltalog_run.argtypes = [i, i, i, i, i, i, d, P, P, P, P, P,
                                                 P, P, P, P, P, P, P, P, P, i]
+            lib.oracle_deltalog_slots_run.argtypes = [i, i, i, i, i, i, i, d, P, P, P, P, P, P,
+                                                      P, P, P, P, P, P, P, P, i]
             lib.oracle_materialize.argtypes = [i, i, i, i, i, i, P, P, P, P, P]
             lib.oracle_merge.argtypes = [i, i, i, i, i, i, P, P, P, P]
             lib.oracle_max_threads.argtypes = []
-            for f in ("oracle_eager_run", "oracle_deltalog_run",
+            for f in ("oracle_eager_run", "oracle_deltalog_run", "oracle_deltalog_slots_run",
                       "oracle_materialize", "oracle_merge", "oracle_max_threads"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
@@ -72,8 +74,8 @@ def _use_library(path):
     if path is None:
         return prev
     lib = ctypes.CDLL(path)
-    for f in ("oracle_eager_run", "oracle_deltalog_run", "oracle_materialize",
-              "oracle_merge", "oracle_max_threads"):
+    for f in ("oracle_eager_run", "oracle_deltalog_run", "oracle_deltalog_slots_run",
+              "oracle_materialize", "oracle_merge", "oracle_max_threads"):
         getattr(lib, f).argtypes = getattr(prev, f).argtypes
         getattr(lib, f).restype = ctypes.c_int
     with _lock:
@@ -187,6 +189,42 @@ def deltalog_run(state: LogState, q, k, v, beta, g, bonus=None, scale=1.0,
         raise ValueError("oracle_deltalog_run rejected its arguments")
     state.L = int(L_io.value)
     return out, L_trace, merged
+
+
+def deltalog_slots_run(state: LogState, H, Ls, active, q, k, v, beta, g, bonus=None,
+                       scale=1.0, n_threads=None):
+    """Base+log decode with a log length per slot: the state's heads are
+    grouped into slots of H heads (head = slot * H + h), slot s takes part in
+    token t only where active[t, s], and each slot appends and merges on its
+    own schedule.  `Ls` (int array, one entry per slot) is advanced in place;
+    state.L is not used.
+
+    Returns (out [T, nh, dv] with NaN rows for idle slots, L_trace [T, nslots]).
+    """
+    op, C = state.op, state.C
+    nh, dk, dv = state.base.shape
+    if nh % H:
+        raise ValueError("heads are not a whole number of slots")
+    nslots = nh // H
+    q = _f64(q); T = q.shape[0]
+    m = decay_width(op, dk)
+    k = _f64(k); v = _f64(v)
+    g = _f64(g, (T, nh, m))
+    beta = _f64(beta, (T, nh)) if beta is not None else np.zeros((T, nh))
+    bonus = _f64(bonus, (nh, dk)) if bonus is not None else (
+        np.zeros((nh, dk)) if op == RWKV6 else None)
+    act = np.ascontiguousarray(np.asarray(active, dtype=bool).reshape(T, nslots), dtype=np.uint8)
+    Ls_c = np.ascontiguousarray(np.asarray(Ls).reshape(nslots), dtype=np.int32).copy()
+    out = np.full((T, nh, dv), np.nan)
+    L_trace = np.zeros((T, nslots), dtype=np.int32)
+    rc = _load().oracle_deltalog_slots_run(
+        op, nslots, H, dk, dv, C, T, float(scale), _p(state.base), _p(state.K), _p(state.U),
+        _p(state.Lam), _p(Ls_c), _p(act), _p(q), _p(k), _p(v), _p(beta), _p(g), _p(bonus),
+        _p(out), _p(L_trace), _threads(n_threads))
+    if rc:
+        raise ValueError("oracle_deltalog_slots_run rejected its arguments")
+    Ls[...] = Ls_c.reshape(np.shape(Ls))
+    return out, L_trace
 
 
 def materialize(state: LogState):

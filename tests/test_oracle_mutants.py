@@ -42,6 +42,9 @@ MUTANTS = {
          "xr += base[(size_t)i * dv + c] * exp(lam_t[i]) * q[i];"),
     "value replay uses key coefficient":
         ("rq += dj[j] * U[(size_t)j * dv + c];", "rq += cj[j] * U[(size_t)j * dv + c];"),
+    "idle slot still decodes":
+        ("if (!active[(size_t)t * nslots + s]) continue;",
+         "if (0 && !active[(size_t)t * nslots + s]) continue;"),
     "merge replays one entry too few":
         ("for (int j = 0; j < L; ++j) s += coef[j] * U[(size_t)j * dv + c];",
          "for (int j = 0; j + 1 < L; ++j) s += coef[j] * U[(size_t)j * dv + c];"),
@@ -60,6 +63,8 @@ PIN_CALLS = [
              for op in (0, 1, 2) for d in ((2, 3), (3, 2))],
     lambda: [pins.test_log_contents(None, op) for op in (0, 1, 2)],
     lambda: [pins.test_merge_properties(None, op) for op in (0, 1, 2)],
+    lambda: [pins.test_slots_match_eager_on_each_slots_tokens(None, op, C)
+             for op in (0, 1, 2) for C in (1, 3)],
 ]
 
 

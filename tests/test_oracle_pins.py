@@ -324,6 +324,75 @@ def test_schedule(oracle_lib, C, L0):
     assert st.L == exp_L[-1]
 
 
+# ---------------------------------------------------- per-slot log lengths --
+
+def _slot_mask(rng, T, nslots, p=0.6):
+    act = rng.random((T, nslots)) < p
+    act[0, :] = True
+    return act
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("C", [1, 2, 3, 5])
+def test_slots_match_eager_on_each_slots_tokens(oracle_lib, op, C):
+    """Continuous batching: every slot, on its own, is the eager recurrence
+    over the tokens it took part in (from the state it had on entry), and its
+    log length counts those tokens modulo C.  Entry lengths differ (a common
+    prefix of 1 or 2 tokens is decoded first), idle slots are not touched."""
+    rng = np.random.default_rng(300 + 10 * op + C)
+    nslots, H, dk, dv, T = 3, 2, 3, 2, 4 * C + 3
+    nh = nslots * H
+    S0 = rng.standard_normal((nh, dk, dv))
+    q, k, v, beta, g, bonus = rand_inputs(rng, op, nh, dk, dv, T + 2)
+    b_ = None if op == RWKV6 else beta
+    st = LogState(op, S0, C)
+    pre = 1 + (C > 2)                                     # common prefix
+    o_pre, _, _ = oracle.deltalog_run(st, q[:pre], k[:pre], v[:pre],
+                                      None if b_ is None else b_[:pre], g[:pre], bonus, 0.6)
+    Ls = np.full(nslots, st.L, dtype=np.int32)
+    act = _slot_mask(rng, T, nslots)
+    sl = slice(pre, pre + T)
+    out, Ltr = oracle.deltalog_slots_run(st, H, Ls, act, q[sl], k[sl], v[sl],
+                                         None if b_ is None else b_[sl], g[sl], bonus, 0.6)
+    for s in range(nslots):
+        hs = slice(s * H, (s + 1) * H)
+        ts = [pre + t for t in range(T) if act[t, s]]
+        idx = list(range(pre)) + ts
+        S_e, o_e = oracle.eager_run(op, S0[hs], q[idx][:, hs], k[idx][:, hs], v[idx][:, hs],
+                                    None if b_ is None else b_[idx][:, hs], g[idx][:, hs],
+                                    None if bonus is None else bonus[hs], 0.6)
+        got = out[[t - pre for t in ts]][:, hs]
+        assert rel_err(got, o_e[pre:]) < TIGHT, s
+        assert np.all(np.isnan(out[~act[:, s]][:, hs])), s
+        mat = oracle.materialize(LogState(op, st.base[hs], C, int(Ls[s]), st.K[hs], st.U[hs],
+                                          st.Lam[hs]))
+        assert rel_err(mat, S_e) < TIGHT, s
+        count = pre + np.cumsum(act[:, s])
+        assert Ltr[:, s].tolist() == (count % C).tolist()
+        assert Ls[s] == count[-1] % C
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_slots_all_active_is_the_shared_schedule(oracle_lib, op):
+    """With every slot active every token the per-slot run is the shared-length
+    run, to the last bit."""
+    rng = np.random.default_rng(77 + op)
+    nslots, H, dk, dv, C, T = 2, 3, 4, 3, 3, 8
+    nh = nslots * H
+    S0 = rng.standard_normal((nh, dk, dv))
+    q, k, v, beta, g, bonus = rand_inputs(rng, op, nh, dk, dv, T)
+    b_ = None if op == RWKV6 else beta
+    a = LogState(op, S0, C, L=1)
+    b = LogState(op, S0, C, L=1)
+    o_a, Ltr, _ = oracle.deltalog_run(a, q, k, v, b_, g, bonus, 0.5)
+    Ls = np.ones(nslots, dtype=np.int32)
+    o_b, Ltr_b = oracle.deltalog_slots_run(b, H, Ls, np.ones((T, nslots), bool), q, k, v, b_, g,
+                                           bonus, 0.5)
+    assert np.array_equal(o_a, o_b)
+    assert np.array_equal(a.base, b.base) and np.array_equal(a.U, b.U)
+    assert np.all(Ltr_b == Ltr[:, None]) and np.all(Ls == a.L)
+
+
 def test_rel_err_definition():
     assert rel_err([1.0, -2.0], [1.0, -2.0]) == 0.0
     assert math.isclose(rel_err([1.1, -2.0], [1.0, -2.0]), 0.05)
