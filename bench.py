@@ -465,6 +465,26 @@ def run_native(args, rank, world, local_rank):
         cyc_sep.close()
         del sep
 
+    # --- continuous batching: the slots at staggered log lengths (slot b
+    #     joined b mod C tokens late), so every token of the cycle runs an
+    #     append over 7/8 of the slots and a merge-token over the rest
+    if args.staggered and C > 1:
+        stag = _layers(w, R, rank, dev, B.DL_MERGE_FOLD)
+        for l, L_ in enumerate(stag):
+            for t in range(C - 1):
+                L_.step(xs[l], t, outs[l][t], stream=stream,
+                        active=[(b % C) > t for b in range(w.B)])
+        cyc_st = B.Cycle([L_.handle for L_ in stag], _ios(w, xs, outs, R, C))
+        ms = _time_graph(lambda: cyc_st.launch(stream), stream, args.steps, args.warmup, dev)
+        ms = ms / args.steps
+        result["staggered"] = {
+            "us_per_token": ms * 1e3 / (C * R),
+            "hbm_gbs": gbs * us_per_token / (ms * 1e3 / (C * R)),
+            "kernels_per_step": cyc_st.kernels,
+            "slot_lengths": "slot b at b mod C when the cycle starts"}
+        cyc_st.close()
+        del stag
+
     # --- eager dense baseline, same layers and rotation, graph-captured
     if args.eager:
         cfg = D.config_of(w)
@@ -571,6 +591,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--no-eager", dest="eager", action="store_false")
+    ap.add_argument("--no-staggered", dest="staggered", action="store_false",
+                    help="skip the cycle with slots at staggered log lengths")
     ap.add_argument("--no-ablation", dest="ablation", action="store_false",
                     help="skip the separate-merge cycle")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")

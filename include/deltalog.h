@@ -131,7 +131,8 @@ dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void 
                          const float *beta, const float *g, void *out, void *stream);
 
 /* Merge phase (paper: "Fase di Merge"): Sbar <- D(exp(Lambda_L)) Sbar +
- * sum_j D(exp(Lambda_L - Lambda_j)) k_j u_j^T in place, then L = 0.
+ * sum_j D(exp(Lambda_L - Lambda_j)) k_j u_j^T in place, then L = 0 (every
+ * slot at its own length L_b; slots at 0 are left as they are).
  * A no-op when L = 0.  Errors: DL_ECUDA. */
 dl_status dl_merge(dl_handle *h, void *stream);
 
@@ -150,8 +151,44 @@ dl_status dl_eager_step(const dl_config *cfg, float *S, const void *q, const voi
                         const void *v, const float *beta, const float *g,
                         const float *bonus, void *out, void *stream);
 
-/* Current log length L (0 <= L <= C), or -1 for a NULL handle. */
+/* The log length L (0 <= L <= C) every slot has, -2 when the slots'
+ * lengths differ (see dl_slot_len), or -1 for a NULL handle. */
 int dl_log_len(const dl_handle *h);
+
+/* --------------------------------------------- per-slot log lengths ---- */
+/* Continuous batching: every slot b (batch row, heads b*H .. b*H + H-1)
+ * keeps its own log length L_b, so sequences can join, leave and idle
+ * independently and each slot merges when its own log is full.  The log of
+ * a (slot, head) pair is the paper's per-"slot-head" unit (gist.science
+ * technical summary, "Implementazione del Kernel": ReplayPrep coefficients
+ * are computed once per slot-head).  All slots start at L_b = 0; while every
+ * slot has the same length and every slot decodes, nothing differs from
+ * the shared-length calls above.  dl_merge folds every slot's log (each at
+ * its own length); dl_materialize writes every slot's logical state. */
+
+/* One decode token for the slots with active[b] != 0 (`active`: host array
+ * of B bytes, read during the call; NULL = every slot).  Each active slot
+ * takes the step dl_decode_step describes at its own length L_b; idle
+ * slots' base, log and output rows are not touched and L_b does not move.
+ * A step launches at most one append kernel (the slots below their last
+ * entry), one merge-token kernel (DL_MERGE_FOLD: the slots at L_b = C-1)
+ * and one merge kernel (DL_MERGE_SEPARATE: the slots that reach C), each
+ * over just its slots (split into launches of at most 512 slots).
+ * Errors: as dl_decode_step; DL_ESTATE if an active slot's log is full
+ * with DL_MERGE_OFF (nothing launched, no length moves). */
+dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const void *q,
+                                const void *k, const void *v, const float *beta,
+                                const float *g, void *out, void *stream);
+
+/* Slot `slot` begins a new sequence: L_slot = 0, so its logged entries are
+ * dropped.  The slot's base rows ([H, d_k, d_v] at head slot*H) are the
+ * caller's to fill with the sequence's starting state (zeros, or the state
+ * a prefill produced) before the next call that reads them.  Host-side
+ * only: nothing is launched.  Errors: DL_EINVAL (NULL handle, bad slot). */
+dl_status dl_slot_reset(dl_handle *h, int slot);
+
+/* Log length of one slot, or -1 for a NULL handle or a slot out of range. */
+int dl_slot_len(const dl_handle *h, int slot);
 
 /* Release the handle (host memory only).  NULL is accepted. */
 void dl_destroy(dl_handle *h);
@@ -166,9 +203,13 @@ void dl_destroy(dl_handle *h);
  *
  * `io` is [C][n_layers] (token-major): the device pointers of each
  * (token, layer) step, laid out as for dl_decode_step.  All layers must have
- * the same C, an automatic merge mode, and L = 0 when the cycle is launched;
- * they are back at L = 0 afterwards.  The graph captures the pointers: new inputs are
- * written into the same buffers between launches. */
+ * the same C and an automatic merge mode.  The cycle decodes C tokens for
+ * every slot starting from the log lengths the layers have at creation
+ * (usually L = 0; with per-slot lengths, every step holds one launch per
+ * kind of step its slots take), after which every length is back where it
+ * started: a launch requires the layers to be in that state.  The graph
+ * captures the pointers: new inputs are written into the same buffers
+ * between launches. */
 typedef struct {
     const void *q, *k, *v;
     const float *beta, *g;
@@ -177,10 +218,11 @@ typedef struct {
 
 typedef struct dl_cycle dl_cycle;
 
-/* Errors: DL_EINVAL (mixed C, bad pointer), DL_ESTATE, DL_ECUDA, DL_ENOMEM. */
+/* Errors: DL_EINVAL (mixed C, DL_MERGE_OFF, bad pointer), DL_ECUDA, DL_ENOMEM. */
 dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_io *io,
                           dl_cycle **out);
-/* Launch one cycle on `stream`.  DL_ESTATE if any layer has L != 0. */
+/* Launch one cycle on `stream`.  DL_ESTATE if any layer's log lengths are
+ * not those the cycle was created at. */
 dl_status dl_cycle_launch(dl_cycle *cy, void *stream);
 /* Kernels in one launch of the cycle. */
 int dl_cycle_kernels(const dl_cycle *cy);

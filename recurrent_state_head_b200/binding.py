@@ -27,6 +27,7 @@ DL_MERGE_OFF, DL_MERGE_FOLD, DL_MERGE_SEPARATE = 0, 1, 2
 EXPORTS = (
     "dl_log_bytes", "dl_log_layout", "dl_create", "dl_decode_step", "dl_merge",
     "dl_materialize", "dl_eager_step", "dl_log_len", "dl_destroy",
+    "dl_decode_step_masked", "dl_slot_reset", "dl_slot_len",
     "dl_cycle_create", "dl_cycle_launch", "dl_cycle_kernels", "dl_cycle_destroy",
     "dl_strerror", "dl_last_error",
 )
@@ -75,6 +76,9 @@ def lib() -> ctypes.CDLL:
             L.dl_materialize.argtypes = [P, P, P]
             L.dl_eager_step.argtypes = [CP, P, P, P, P, P, P, P, P, P]
             L.dl_log_len.argtypes, L.dl_log_len.restype = [P], I
+            L.dl_decode_step_masked.argtypes = [P, P, P, P, P, P, P, P, P]
+            L.dl_slot_reset.argtypes = [P, I]
+            L.dl_slot_len.argtypes, L.dl_slot_len.restype = [P, I], I
             L.dl_destroy.argtypes, L.dl_destroy.restype = [P], None
             L.dl_cycle_create.argtypes = [ctypes.POINTER(P), I, ctypes.POINTER(dl_step_io),
                                           ctypes.POINTER(P)]
@@ -146,6 +150,24 @@ def dl_decode_step(h: int, q, k, v, beta, g, out, stream=None):
                                 _ptr(out), _stream(stream)))
 
 
+def dl_decode_step_masked(h: int, active, q, k, v, beta, g, out, stream=None):
+    """`active`: None (every slot) or a sequence of B truth values (host)."""
+    act = None
+    if active is not None:
+        flags = bytes(1 if a else 0 for a in active)
+        act = ctypes.create_string_buffer(flags, len(flags))
+    _check(lib().dl_decode_step_masked(h, act, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g),
+                                       _ptr(out), _stream(stream)))
+
+
+def dl_slot_reset(h: int, slot: int):
+    _check(lib().dl_slot_reset(h, int(slot)))
+
+
+def dl_slot_len(h: int, slot: int) -> int:
+    return int(lib().dl_slot_len(h, int(slot)))
+
+
 def dl_merge(h: int, stream=None):
     _check(lib().dl_merge(h, _stream(stream)))
 
@@ -214,8 +236,17 @@ class Handle:
     def L(self) -> int:
         return dl_log_len(self.h)
 
-    def decode_step(self, q, k, v, beta, g, out, stream=None):
-        dl_decode_step(self.h, q, k, v, beta, g, out, stream)
+    def decode_step(self, q, k, v, beta, g, out, stream=None, active=None):
+        if active is None:
+            dl_decode_step(self.h, q, k, v, beta, g, out, stream)
+        else:
+            dl_decode_step_masked(self.h, active, q, k, v, beta, g, out, stream)
+
+    def slot_len(self, slot: int) -> int:
+        return dl_slot_len(self.h, slot)
+
+    def slot_reset(self, slot: int):
+        dl_slot_reset(self.h, slot)
 
     def merge(self, stream=None):
         dl_merge(self.h, stream)

@@ -1,0 +1,101 @@
+// append_launch.cuh -- internal: launch templates of the append + read-out
+// kernel and its merge-token variant, for one log length shared by every
+// head (append_kernel) or a list of slots with their own lengths
+// (append_slots_kernel).
+#pragma once
+
+#include "launch.h"
+
+namespace dl {
+namespace append_detail {
+
+// Plain launch, or a programmatic dependent launch when p.early (it may
+// start while the previous kernel of the stream finishes; the kernel orders
+// itself with griddepcontrol).
+template <typename Kernel, typename... Args>
+cudaError_t launch_kernel(Kernel kern, unsigned grid, int threads, size_t smem, bool early,
+                          cudaStream_t s, const Args &...args) {
+    if (!early) {
+        kern<<<grid, threads, smem, s>>>(args...);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <int OP, int DK, int DV, int TV, bool FOLD, int LB>
+cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
+    constexpr int NT = CtaShape<DK, TV>::NT;
+    static std::atomic<unsigned long long> smem_ok{0};
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB>;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((long long)p.NH * (DV / TV));
+    return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p);
+}
+
+// The merge-token keeps the logged value factors in registers while the log
+// is short; longer logs are read from shared memory.  The merge-token sees
+// L = C - 1, so the buckets end at 3 and 7 (C = 4 and C = 8 without padding).
+template <int OP, int DK, int DV, int TV, bool FOLD>
+cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
+    if constexpr (FOLD) {
+        if (p.L <= 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
+        if (p.L <= 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
+    }
+    return launch_lb<OP, DK, DV, TV, FOLD, 0>(p, s);
+}
+
+template <int OP, int DK, int DV, bool FOLD>
+cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    switch (pick_tile(p.NH, DV, sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, FOLD>(p, s); break;
+        case 64: return launch_tv<OP, DK, DV, 64, FOLD>(p, s);
+        default: break;
+    }
+    return launch_tv<OP, DK, DV, 32, FOLD>(p, s);
+}
+
+// Slot list: p.L is the longest length in the list.
+template <int OP, int DK, int DV, int TV>
+cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+    constexpr int NT = CtaShape<DK, TV>::NT;
+    static std::atomic<unsigned long long> smem_ok{0};
+    auto kern = append_slots_kernel<OP, DK, DV, TV, NT>;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, sl.nfold > 0).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, true).bytes);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((long long)sl.n * p.H * (DV / TV));
+    return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p, sl);
+}
+
+template <int OP, int DK, int DV>
+cudaError_t launch_slots(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    switch (pick_tile((long long)sl.n * p.H, DV, sms)) {
+        case 128: if constexpr (DV >= 128) return launch_slots_tv<OP, DK, DV, 128>(p, sl, s); break;
+        case 64: return launch_slots_tv<OP, DK, DV, 64>(p, sl, s);
+        default: break;
+    }
+    return launch_slots_tv<OP, DK, DV, 32>(p, sl, s);
+}
+
+}  // namespace append_detail
+}  // namespace dl

@@ -95,13 +95,49 @@ dl_status check_step_ptrs(const dl_config *c, const void *q, const void *k, cons
 
 }  // namespace
 
+namespace {
+
+// Log lengths of a handle's slots: one shared length while every slot has
+// it (the common case), else one length per slot.
+struct Lens {
+    bool shared = true;
+    int L = 0;                          // the shared length
+    std::vector<unsigned char> per;     // per-slot lengths when !shared
+
+    int of(int b) const { return shared ? L : per[(size_t)b]; }
+    // Expand to per-slot form (B slots).
+    void split(int B) {
+        if (!shared) return;
+        per.assign((size_t)B, (unsigned char)L);
+        shared = false;
+    }
+    // Back to the shared form when every slot has the same length.
+    void join() {
+        if (shared || per.empty()) return;
+        for (unsigned char x : per)
+            if (x != per[0]) return;
+        L = per[0];
+        shared = true;
+        per.clear();
+    }
+    bool operator==(const Lens &o) const {
+        if (shared && o.shared) return L == o.L;
+        const size_t n = shared ? o.per.size() : per.size();
+        for (size_t b = 0; b < n; ++b)
+            if (of((int)b) != o.of((int)b)) return false;
+        return true;
+    }
+};
+
+}  // namespace
+
 struct dl_handle {
     dl_config cfg;
     float *base;
     char *log;
     Layout lay;
     const float *bonus;
-    int L;
+    Lens lens;
     int NH;
 };
 
@@ -109,6 +145,7 @@ struct dl_cycle {
     cudaGraph_t graph;
     cudaGraphExec_t exec;
     std::vector<dl_handle *> layers;
+    std::vector<Lens> start;            // the layers' lengths the cycle starts (and ends) at
     int kernels;
 };
 
@@ -146,6 +183,7 @@ dl::MergeParams merge_params(const dl_handle *h, float *dst, int L) {
     p.logU = h->log + h->lay.U;
     p.logLam = reinterpret_cast<const float *>(h->log + h->lay.Lam);
     p.NH = h->NH;
+    p.H = h->cfg.H;
     p.C = h->cfg.C;
     p.L = L;
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
@@ -182,6 +220,109 @@ bool disjoint_bases(dl_handle *const *layers, int n) {
 cudaError_t launch_merge(const dl_handle *h, float *dst, int L, cudaStream_t s) {
     if (h->NH == 0) return cudaSuccess;
     return dl::get_merge(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, L), s);
+}
+
+// Slot-list launches of at most MAXSEL slots each: `ids` are the slots,
+// `lens` their lengths.  merge == false: the append kernel, whose first
+// `nfold` entries take the merge-token; merge == true: the merge kernel into
+// dst.
+cudaError_t launch_slots(const dl_handle *h, bool merge, const std::vector<int> &ids,
+                         const std::vector<int> &lens, int nfold, const dl_step_io *io, float *dst,
+                         cudaStream_t s, bool early, int *kernels) {
+    if (h->NH == 0) return cudaSuccess;
+    for (size_t at = 0; at < ids.size(); at += dl::MAXSEL) {
+        const size_t n = ids.size() - at < (size_t)dl::MAXSEL ? ids.size() - at : (size_t)dl::MAXSEL;
+        dl::SlotList sl;
+        sl.n = (int)n;
+        const int fold_left = nfold - (int)at;
+        sl.nfold = fold_left <= 0 ? 0 : (fold_left < (int)n ? fold_left : (int)n);
+        int Lmax = 0;
+        for (size_t i = 0; i < n; ++i) {
+            sl.id[i] = (unsigned short)ids[at + i];
+            sl.L[i] = (unsigned char)lens[at + i];
+            if (lens[at + i] > Lmax) Lmax = lens[at + i];
+        }
+        cudaError_t e;
+        if (merge) {
+            e = dl::get_merge_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, Lmax), sl, s);
+        } else {
+            dl::AppendParams p = append_params(h, *io, Lmax);
+            p.early = early ? 1 : 0;
+            e = dl::get_append_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, sl, s);
+        }
+        if (e != cudaSuccess) return e;
+        if (kernels) *kernels += 1;
+    }
+    return cudaSuccess;
+}
+
+// One decode token for the active slots (active == nullptr: all of them),
+// launched on `st`, with the lengths in `ln` (advanced on success).
+// Returns DL_OK, DL_ESTATE (nothing launched) or DL_ECUDA (lengths unchanged).
+dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active, const dl_step_io &io,
+                      cudaStream_t st, bool early, int *kernels) {
+    const int B = h->cfg.B, C = h->cfg.C, mode = h->cfg.auto_merge;
+    bool all = true;
+    if (active)
+        for (int b = 0; b < B && all; ++b) all = active[b] != 0;
+    if (ln.shared && all) {
+        if (ln.L >= C)
+            return fail(DL_ESTATE, "log is full (L = C = %d) and auto_merge is off: merge first", C);
+        if (mode == DL_MERGE_FOLD && ln.L == C - 1) {
+            // the token that completes the log: one kernel reads the base once
+            // and writes the merged logical state back
+            cudaError_t e = launch_append(h, io, ln.L, true, st, early);
+            if (e != cudaSuccess) return cuda_fail(e, "merge-token kernel launch");
+            if (kernels && h->NH > 0) *kernels += 1;
+            ln.L = 0;
+            return ok();
+        }
+        cudaError_t e = launch_append(h, io, ln.L, false, st, early);
+        if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+        if (kernels && h->NH > 0) *kernels += 1;
+        ln.L += 1;
+        if (mode == DL_MERGE_SEPARATE && ln.L == C) {
+            e = launch_merge(h, h->base, ln.L, st);
+            if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
+            if (kernels && h->NH > 0) *kernels += 1;
+            ln.L = 0;
+        }
+        return ok();
+    }
+    // slots at different lengths, or some idle: one append launch over the
+    // active slots, merge-token slots (DL_MERGE_FOLD, log one short of full)
+    // first; with DL_MERGE_SEPARATE the slots that fill their log are then
+    // merged by the merge kernel
+    std::vector<int> ids, lens, idm, lm;
+    int nfold = 0;
+    for (int pass = 0; pass < 2; ++pass)
+        for (int b = 0; b < B; ++b) {
+            if (active && !active[b]) continue;
+            const int L = ln.of(b);
+            if (L >= C)
+                return fail(DL_ESTATE, "slot %d's log is full (L = C = %d) and auto_merge is off: merge first",
+                            b, C);
+            const bool fold = mode == DL_MERGE_FOLD && L == C - 1;
+            if (fold != (pass == 0)) continue;
+            ids.push_back(b);
+            lens.push_back(L);
+            nfold += fold ? 1 : 0;
+            if (mode == DL_MERGE_SEPARATE && L + 1 == C) {
+                idm.push_back(b);
+                lm.push_back(C);
+            }
+        }
+    cudaError_t e = launch_slots(h, false, ids, lens, nfold, &io, nullptr, st, early, kernels);
+    if (e == cudaSuccess) e = launch_slots(h, true, idm, lm, 0, nullptr, h->base, st, false, kernels);
+    if (e != cudaSuccess) return cuda_fail(e, "per-slot kernel launch");
+    ln.split(B);
+    for (int b = 0; b < B; ++b) {
+        if (active && !active[b]) continue;
+        const int L = ln.per[(size_t)b] + 1;
+        ln.per[(size_t)b] = (unsigned char)((mode != DL_MERGE_OFF && L == C) ? 0 : L);
+    }
+    ln.join();
+    return ok();
 }
 
 }  // namespace
@@ -224,48 +365,50 @@ dl_status dl_create(const dl_config *cfg, float *base, void *log_ws, const float
     h->log = static_cast<char *>(log_ws);
     h->lay = log_layout(cfg);
     h->bonus = cfg->op == DL_RWKV6 ? bonus : nullptr;
-    h->L = 0;
     h->NH = NH;
     *out = h;
     return ok();
 }
 
-dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
-                         const float *beta, const float *g, void *out, void *stream) {
+dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const void *q,
+                                const void *k, const void *v, const float *beta,
+                                const float *g, void *out, void *stream) {
     if (!h) return fail(DL_EINVAL, "handle is NULL");
     if (h->NH > 0) {
         dl_status s = check_step_ptrs(&h->cfg, q, k, v, beta, g, out);
         if (s != DL_OK) return s;
     }
-    if (h->L >= h->cfg.C)
-        return fail(DL_ESTATE, "log is full (L = C = %d) and auto_merge is off: merge first", h->cfg.C);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const dl_step_io io = {q, k, v, beta, g, out};
-    if (h->cfg.auto_merge == DL_MERGE_FOLD && h->L == h->cfg.C - 1) {
-        // the token that completes the log: one kernel reads the base once
-        // and writes the merged logical state back
-        cudaError_t e = launch_append(h, io, h->L, true, st);
-        if (e != cudaSuccess) return cuda_fail(e, "merge-token kernel launch");
-        h->L = 0;
-        return ok();
-    }
-    cudaError_t e = launch_append(h, io, h->L, false, st);
-    if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
-    h->L += 1;
-    if (h->cfg.auto_merge == DL_MERGE_SEPARATE && h->L == h->cfg.C) {
-        e = launch_merge(h, h->base, h->L, st);
-        if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
-        h->L = 0;
-    }
-    return ok();
+    Lens ln = h->lens;
+    dl_status s = decode_step(h, ln, active, io, static_cast<cudaStream_t>(stream), false, nullptr);
+    if (s == DL_OK) h->lens = std::move(ln);
+    return s;
+}
+
+dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
+                         const float *beta, const float *g, void *out, void *stream) {
+    return dl_decode_step_masked(h, nullptr, q, k, v, beta, g, out, stream);
 }
 
 dl_status dl_merge(dl_handle *h, void *stream) {
     if (!h) return fail(DL_EINVAL, "handle is NULL");
-    if (h->L == 0) return ok();
-    cudaError_t e = launch_merge(h, h->base, h->L, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (h->lens.shared) {
+        if (h->lens.L == 0) return ok();
+        cudaError_t e = launch_merge(h, h->base, h->lens.L, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
+        h->lens.L = 0;
+        return ok();
+    }
+    std::vector<int> ids, lens;
+    for (int b = 0; b < h->cfg.B; ++b)
+        if (h->lens.of(b) > 0) {
+            ids.push_back(b);
+            lens.push_back(h->lens.of(b));
+        }
+    cudaError_t e = launch_slots(h, true, ids, lens, 0, nullptr, h->base, st, false, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
-    h->L = 0;
+    h->lens = Lens();
     return ok();
 }
 
@@ -276,7 +419,18 @@ dl_status dl_materialize(const dl_handle *h, float *S_out, void *stream) {
     const size_t bytes = (size_t)h->NH * h->cfg.dk * h->cfg.dv * 4;
     const char *a = reinterpret_cast<const char *>(S_out), *b = reinterpret_cast<const char *>(h->base);
     if (a < b + bytes && b < a + bytes) return fail(DL_EINVAL, "S_out overlaps the base state");
-    cudaError_t e = launch_merge(h, S_out, h->L, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (h->lens.shared) {
+        e = launch_merge(h, S_out, h->lens.L, st);
+    } else {
+        std::vector<int> ids, lens;
+        for (int b = 0; b < h->cfg.B; ++b) {
+            ids.push_back(b);
+            lens.push_back(h->lens.of(b));
+        }
+        e = launch_slots(h, true, ids, lens, 0, nullptr, S_out, st, false, nullptr);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "materialize kernel launch");
     return ok();
 }
@@ -312,7 +466,25 @@ dl_status dl_eager_step(const dl_config *cfg, float *S, const void *q, const voi
     return ok();
 }
 
-int dl_log_len(const dl_handle *h) { return h ? h->L : -1; }
+int dl_log_len(const dl_handle *h) {
+    if (!h) return -1;
+    return h->lens.shared ? h->lens.L : -2;
+}
+
+dl_status dl_slot_reset(dl_handle *h, int slot) {
+    if (!h) return fail(DL_EINVAL, "handle is NULL");
+    if (slot < 0 || slot >= h->cfg.B) return fail(DL_EINVAL, "slot %d outside [0, %d)", slot, h->cfg.B);
+    if (h->lens.of(slot) == 0) return ok();
+    h->lens.split(h->cfg.B);
+    h->lens.per[(size_t)slot] = 0;
+    h->lens.join();
+    return ok();
+}
+
+int dl_slot_len(const dl_handle *h, int slot) {
+    if (!h || slot < 0 || slot >= h->cfg.B) return -1;
+    return h->lens.of(slot);
+}
 
 void dl_destroy(dl_handle *h) { delete h; }
 
@@ -327,7 +499,6 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
         if (!h) return fail(DL_EINVAL, "layer %d is NULL", l);
         if (h->cfg.C != C) return fail(DL_EINVAL, "layers must share one log capacity C");
         if (h->cfg.auto_merge == DL_MERGE_OFF) return fail(DL_EINVAL, "layer %d has auto_merge = 0", l);
-        if (h->L != 0) return fail(DL_ESTATE, "layer %d has L = %d, a cycle starts at L = 0", l, h->L);
         for (int t = 0; t < C; ++t) {
             const dl_step_io &x = io[(size_t)t * n_layers + l];
             if (h->NH > 0) {
@@ -343,6 +514,7 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
     cy->kernels = 0;
     try {
         cy->layers.assign(layers, layers + n_layers);
+        for (int l = 0; l < n_layers; ++l) cy->start.push_back(layers[l]->lens);
     } catch (...) {
         delete cy;
         return fail(DL_ENOMEM, "host allocation of the cycle failed");
@@ -358,29 +530,27 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
         return cuda_fail(e, "capture stream creation");
     }
     e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
-    cudaError_t le = cudaSuccess;
+    dl_status ls = DL_OK;
     if (e == cudaSuccess) {
-        // token-major: every layer's step for token t; the token that
-        // completes a layer's log is its merge-token (DL_MERGE_FOLD) or its
-        // append followed by its merge (DL_MERGE_SEPARATE)
-        for (int t = 0; t < C && le == cudaSuccess; ++t) {
-            for (int l = 0; l < n_layers && le == cudaSuccess; ++l) {
-                const dl_handle *h = layers[l];
-                const bool last = t == C - 1;
-                const bool fold = last && h->cfg.auto_merge == DL_MERGE_FOLD;
-                le = launch_append(h, io[(size_t)t * n_layers + l], t, fold, st, overlap);
-                if (h->NH > 0) cy->kernels += 1;
-                if (le == cudaSuccess && last && h->cfg.auto_merge == DL_MERGE_SEPARATE) {
-                    le = launch_merge(h, h->base, C, st);
-                    if (h->NH > 0) cy->kernels += 1;
-                }
-            }
-        }
+        // token-major: every layer's step for token t, on copies of the
+        // layers' lengths (C steps bring every length back where it started);
+        // the token that completes a log is its merge-token (DL_MERGE_FOLD)
+        // or its append followed by its merge (DL_MERGE_SEPARATE)
+        std::vector<Lens> lens(cy->start);
+        for (int t = 0; t < C && ls == DL_OK; ++t)
+            for (int l = 0; l < n_layers && ls == DL_OK; ++l)
+                ls = decode_step(layers[l], lens[(size_t)l], nullptr, io[(size_t)t * n_layers + l], st,
+                                 overlap, &cy->kernels);
         cudaGraph_t g = nullptr;
         e = cudaStreamEndCapture(st, &g);
         cy->graph = g;
     }
-    if (e == cudaSuccess && le != cudaSuccess) e = le;
+    if (e == cudaSuccess && ls != DL_OK) {
+        if (cy->graph) cudaGraphDestroy(cy->graph);
+        cudaStreamDestroy(st);
+        delete cy;
+        return ls;
+    }
     if (e == cudaSuccess) e = cudaGraphInstantiate(&cy->exec, cy->graph, 0);
     cudaStreamDestroy(st);
     if (e != cudaSuccess) {
@@ -395,8 +565,8 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
 dl_status dl_cycle_launch(dl_cycle *cy, void *stream) {
     if (!cy) return fail(DL_EINVAL, "cycle is NULL");
     for (size_t l = 0; l < cy->layers.size(); ++l)
-        if (cy->layers[l]->L != 0)
-            return fail(DL_ESTATE, "layer %zu has L = %d, a cycle starts at L = 0", l, cy->layers[l]->L);
+        if (!(cy->layers[l]->lens == cy->start[l]))
+            return fail(DL_ESTATE, "layer %zu's log lengths are not those the cycle starts at", l);
     cudaError_t e = cudaGraphLaunch(cy->exec, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "merge-cycle graph launch");
     return ok();

@@ -21,6 +21,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace dl {
 
 constexpr int OP_GDN = 0, OP_KDA = 1, OP_RWKV6 = 2;
@@ -53,9 +55,39 @@ struct MergeParams {
     const void *logK;
     const void *logU;
     const float *logLam;
-    int NH, C, L;
+    int NH, H, C, L;
     int in_bf16;
 };
+
+// The slots of one launch when log lengths differ between slots (continuous
+// batching): list entry i is slot id[i] -- heads id[i] * H .. id[i] * H + H - 1
+// -- at log length L[i].  The grid then covers n * H heads instead of all NH,
+// and every head-indexed address (base, log, inputs, output) goes through
+// the list.  Merge launches with one shared length take NoSlots instead.
+constexpr int MAXSEL = 512;
+struct SlotList {
+    int n;
+    int nfold;                       // append kernel: entries [0, nfold) take the merge-token
+    unsigned short id[MAXSEL];
+    unsigned char L[MAXSEL];
+};
+struct NoSlots {};
+template <bool SLOTS>
+using SlotArg = typename std::conditional<SLOTS, SlotList, NoSlots>::type;
+
+// Head index (in [0, NH)) and log length of launch-local head `lh`.
+template <bool SLOTS>
+__device__ __forceinline__ void slot_head(const SlotArg<SLOTS> &sl, int lh, int H, int L0,
+                                          int &head, int &L) {
+    if constexpr (SLOTS) {
+        const int i = lh / H;
+        head = (int)sl.id[i] * H + (lh - i * H);
+        L = sl.L[i];
+    } else {
+        head = lh;
+        L = L0;
+    }
+}
 
 struct EagerParams {
     float *S;                 // [NH, DK, DV] read and rewritten
@@ -131,6 +163,78 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
     const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
+}
+
+// L2 eviction priorities (createpolicy + .L2::cache_hint), used by the
+// append kernel: the read-once base stream is marked evict-first, so that it
+// does not push out of L2 what the next decode token reads again -- the log
+// entries, written and read evict-last while the log is live.  The
+// merge-token reads and writes everything evict-first (its log is dropped).
+// Measured on B200 in a four-layer merge cycle: 1.4 % (GDN) to 3.7 %
+// (RWKV6) faster than without hints; the merge kernel, whose every byte is
+// touched once, is faster without them and uses none.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ float4 ld_stream_hint(const float *p, uint64_t pol) {
+    float4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p), "l"(pol));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_state_hint(const float *p, uint64_t pol) {
+    float4 r;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p), "l"(pol)
+                 : "memory");
+    return r;
+}
+
+__device__ __forceinline__ void st_state_hint(float *p, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_f32_hint(float *p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_b16_hint(void *p, uint16_t v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p), "h"(v), "l"(pol) : "memory");
+}
+
+// element copy into the log (input dtype), with an L2 policy
+__device__ __forceinline__ void copy_raw_hint(void *dst, size_t di, const void *src, int si, int bf16,
+                                              uint64_t pol) {
+    if (bf16)
+        st_b16_hint(reinterpret_cast<uint16_t *>(dst) + di, reinterpret_cast<const uint16_t *>(src)[si], pol);
+    else
+        st_f32_hint(reinterpret_cast<float *>(dst) + di, reinterpret_cast<const float *>(src)[si], pol);
+}
+
+__device__ __forceinline__ void cp_async16_hint(void *smem, const void *gmem, uint64_t pol) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async4_hint(void *smem, const void *gmem, uint64_t pol) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;" ::"r"(sa), "l"(gmem), "l"(pol)
+                 : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait_all() {
@@ -255,6 +359,28 @@ __device__ __forceinline__ void warp_copy(unsigned char *dst, const void *src, i
     for (int o = lane * 16; o < bytes; o += 32 * 16) cp_async16(dst + o, g + o);
 }
 
+// cp.async of 16 / 4 bytes with an L2 policy (HINT) or without one
+template <bool HINT>
+__device__ __forceinline__ void cp16(void *smem, const void *gmem, uint64_t pol) {
+    if constexpr (HINT)
+        cp_async16_hint(smem, gmem, pol);
+    else
+        cp_async16(smem, gmem);
+}
+template <bool HINT>
+__device__ __forceinline__ void cp4(void *smem, const void *gmem, uint64_t pol) {
+    if constexpr (HINT)
+        cp_async4_hint(smem, gmem, pol);
+    else
+        cp_async4(smem, gmem);
+}
+template <bool HINT>
+__device__ __forceinline__ void warp_copy_pol(unsigned char *dst, const void *src, int bytes, int lane,
+                                              uint64_t pol) {
+    const char *g = static_cast<const char *>(src);
+    for (int o = lane * 16; o < bytes; o += 32 * 16) cp16<HINT>(dst + o, g + o, pol);
+}
+
 // Sources of one head's staged operands.
 struct OpSources {
     const void *k, *q, *v;          // token rows (NULL: not staged)
@@ -263,10 +389,12 @@ struct OpSources {
     const float *logLam;
 };
 
-// Stage one unit's operands (warp 0 only), then wait for them.
-template <int OP, int DK, int DV, int TV>
+// Stage one unit's operands (warp 0 only), then wait for them.  The log
+// entries are read with the L2 policy log_pol when HINT is set.
+template <int OP, int DK, int DV, int TV, bool HINT>
 __device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay, const OpSources &src,
-                                          int head, int vt, int L, int C, int H, int ie, bool token) {
+                                          int head, int vt, int L, int C, int H, int ie, bool token,
+                                          uint64_t log_pol) {
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     const int ue = (OP == OP_RWKV6) ? ie : 4;
     const int lane = threadIdx.x & 31;
@@ -285,19 +413,19 @@ __device__ __forceinline__ void stage_ops(unsigned char *sm, const OpLayout &lay
         else if (lane == 1)
             cp_async4(sm + lay.beta, src.beta + head);
     }
-    warp_copy(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie, L * DK * ie,
-              lane);
+    warp_copy_pol<HINT>(sm + lay.K, static_cast<const char *>(src.logK) + (size_t)head * C * DK * ie,
+                        L * DK * ie, lane, log_pol);
     const float *lamh = src.logLam + (size_t)head * C * M;
     if (OP == OP_GDN) {
-        for (int j = lane; j < L; j += 32) cp_async4(sm + lay.lam + 4 * j, lamh + j);
+        for (int j = lane; j < L; j += 32) cp4<HINT>(sm + lay.lam + 4 * j, lamh + j, log_pol);
     } else {
-        warp_copy(sm + lay.lam, lamh, L * DK * 4, lane);
+        warp_copy_pol<HINT>(sm + lay.lam, lamh, L * DK * 4, lane, log_pol);
     }
     const char *lU = static_cast<const char *>(src.logU) + ((size_t)head * C * DV + vt * TV) * ue;
     const int cpr = TV * ue / 16;
     for (int idx = lane; idx < L * cpr; idx += 32) {
         const int j = idx / cpr, c = idx - j * cpr;
-        cp_async16(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16);
+        cp16<HINT>(sm + lay.U + j * TV * ue + c * 16, lU + (size_t)j * DV * ue + c * 16, log_pol);
     }
     cp_async_wait_all();
 }
@@ -387,9 +515,15 @@ __device__ __forceinline__ float4 fold_row_reg(float4 s, float gm, const float *
 //   all L logged factors and this token's k u^T -- is written over the base
 //   tile (the register tile is read once and written once); the log is left
 //   for the caller to reset (L = 0).
-template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0>
-__global__ void __launch_bounds__(NT)
-append_kernel(const AppendParams p) {
+//
+// append_unit does one unit (head, value tile vt) at log length L;
+// append_kernel runs it over all heads at the shared length p.L, and
+// append_slots_kernel over a slot list whose first nfold entries take the
+// merge-token and the rest the append (one launch per step however the
+// slots' lengths are spread).
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB>
+__device__ __forceinline__ void append_unit(const AppendParams &p, const int head, const int vt,
+                                            const int L) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
@@ -409,10 +543,8 @@ append_kernel(const AppendParams p) {
     __shared__ float s_x[NA * TV];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
-    const int unit = blockIdx.x;
-    const int head = unit / T::NVT, vt = unit - head * T::NVT;
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C;
+    const int C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
@@ -424,12 +556,13 @@ append_kernel(const AppendParams p) {
     //    finished; everything else this kernel reads or writes comes after
     //    griddepcontrol.wait (a no-op for an ordinary launch).
     float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+    const uint64_t pol_first = l2_evict_first(), pol_last = l2_evict_last();
     float4 s[T::RPT];
     auto load_base = [&]() {
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r)
-            s[r] = FOLD ? ld_state(bh + (size_t)(rg + r * T::RG) * DV)
-                        : ld_stream(bh + (size_t)(rg + r * T::RG) * DV);
+            s[r] = FOLD ? ld_state_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first)
+                        : ld_stream_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first);
     };
     if (p.early) load_base();
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -439,7 +572,8 @@ append_kernel(const AppendParams p) {
     // 2. small operands, staged by warp 0 while the base loads are in flight
     if (tid < 32) {
         const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
-        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, p.H, ie, true);
+        stage_ops<OP, DK, DV, TV, true>(dsm, lay, src, head, vt, L, C, p.H, ie, true,
+                                        FOLD ? pol_first : pol_last);
     }
     __syncthreads();
     const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
@@ -467,8 +601,8 @@ append_kernel(const AppendParams p) {
             s_w[NA - 1][i] = gam * qf;
         }
         if (!FOLD && vt == 0) {
-            copy_raw(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16);
-            if (OP != OP_GDN || i == 0) p.logLam[((size_t)head * C + L) * M + x] = lt;
+            copy_raw_hint(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16, pol_last);
+            if (OP != OP_GDN || i == 0) st_f32_hint(p.logLam + ((size_t)head * C + L) * M + x, lt, pol_last);
         }
     }
     __syncthreads();
@@ -542,7 +676,7 @@ append_kernel(const AppendParams p) {
             if (FOLD)
                 s_u[c] = vv;
             else
-                copy_raw(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16);
+                copy_raw_hint(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16, pol_last);
         } else {
             const float *U = reinterpret_cast<const float *>(dsm + lay.U);
             float rk = 0.f, rq = 0.f;
@@ -558,7 +692,7 @@ append_kernel(const AppendParams p) {
             if (FOLD)
                 s_u[c] = u;
             else
-                reinterpret_cast<float *>(p.logU)[ub + (size_t)L * DV] = u;
+                st_f32_hint(reinterpret_cast<float *>(p.logU) + ub + (size_t)L * DV, u, pol_last);
         }
     }
 
@@ -580,7 +714,7 @@ append_kernel(const AppendParams p) {
                 const int row = rg + r * T::RG;
                 float4 o = fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L);
                 fma4(o, s_k[row], u4);
-                st_state(bh + (size_t)row * DV, o);
+                st_state_hint(bh + (size_t)row * DV, o, pol_first);
             }
         } else {
 #pragma unroll
@@ -588,10 +722,35 @@ append_kernel(const AppendParams p) {
                 const int row = rg + r * T::RG;
                 float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
                 fma4(o, s_k[row], u4);
-                st_state(bh + (size_t)row * DV, o);
+                st_state_hint(bh + (size_t)row * DV, o, pol_first);
             }
         }
     }
+}
+
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0>
+__global__ void __launch_bounds__(NT)
+append_kernel(const AppendParams p) {
+    using T = Tile<DK, DV, TV, NT>;
+    const int lh = (int)blockIdx.x / T::NVT;
+    append_unit<OP, DK, DV, TV, NT, FOLD, LB>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
+}
+
+// The merge-token entries come first, so that their longer CTAs start in
+// the first wave rather than in the tail.  Both paths read the logged value
+// factors from shared memory (LB = 0) and the kernel is held to the
+// append's 64 registers, so that it keeps the append's occupancy.
+template <int OP, int DK, int DV, int TV, int NT>
+__global__ void __launch_bounds__(NT, 65536 / (NT * 64))
+append_slots_kernel(const AppendParams p, const SlotList sl) {
+    using T = Tile<DK, DV, TV, NT>;
+    const int lh = (int)blockIdx.x / T::NVT, vt = (int)blockIdx.x - lh * T::NVT;
+    const int i = lh / p.H;
+    const int head = (int)sl.id[i] * p.H + (lh - i * p.H);
+    if (i < sl.nfold)
+        append_unit<OP, DK, DV, TV, NT, true, 0>(p, head, vt, sl.L[i]);
+    else
+        append_unit<OP, DK, DV, TV, NT, false, 0>(p, head, vt, sl.L[i]);
 }
 
 // ================================================= merge / materialise ==
@@ -601,9 +760,9 @@ append_kernel(const AppendParams p) {
 // (dst == base) it is the merge; into another buffer it is materialise.
 // One CTA per unit; the register tile is loaded first, the log staged by
 // warp 0, the replay-factor table built once per CTA.
-template <int OP, int DK, int DV, int TV, int NT, int LB = 0>
+template <int OP, int DK, int DV, int TV, int NT, int LB = 0, bool SLOTS = false>
 __global__ void __launch_bounds__(NT)
-merge_kernel(const MergeParams p) {
+merge_kernel(const MergeParams p, const SlotArg<SLOTS> sl) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
 
@@ -612,9 +771,11 @@ merge_kernel(const MergeParams p) {
     __shared__ float s_lL[M];
 
     const int unit = blockIdx.x;
-    const int head = unit / T::NVT, vt = unit - head * T::NVT;
+    const int lh = unit / T::NVT, vt = unit - lh * T::NVT;
+    int head, L;
+    slot_head<SLOTS>(sl, lh, p.H, p.L, head, L);
     const int tid = threadIdx.x;
-    const int L = p.L, C = p.C;
+    const int C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
@@ -628,7 +789,7 @@ merge_kernel(const MergeParams p) {
 
     if (tid < 32) {
         const OpSources src{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, p.logK, p.logU, p.logLam};
-        stage_ops<OP, DK, DV, TV>(dsm, lay, src, head, vt, L, C, 1, ie, false);
+        stage_ops<OP, DK, DV, TV, false>(dsm, lay, src, head, vt, L, C, 1, ie, false, 0);
     }
     __syncthreads();
     const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);

@@ -14,10 +14,18 @@ using append_fn = cudaError_t (*)(const AppendParams &, bool fold, cudaStream_t)
 using merge_fn = cudaError_t (*)(const MergeParams &, cudaStream_t);
 using eager_fn = cudaError_t (*)(const EagerParams &, cudaStream_t);
 
+// The same over a list of slots, each at its own log length; p.L is the
+// longest length in the list.  In the append list, entries [0, nfold) take
+// the merge-token.
+using append_slots_fn = cudaError_t (*)(const AppendParams &, const SlotList &, cudaStream_t);
+using merge_slots_fn = cudaError_t (*)(const MergeParams &, const SlotList &, cudaStream_t);
+
 // Return the launcher for (op, dk, dv), or nullptr for an unsupported shape.
 append_fn get_append(int op, int dk, int dv);
 merge_fn get_merge(int op, int dk, int dv);
 eager_fn get_eager(int op, int dk, int dv);
+append_slots_fn get_append_slots(int op, int dk, int dv);
+merge_slots_fn get_merge_slots(int op, int dk, int dv);
 
 // Number of SMs of the current device (cached per device).
 cudaError_t sm_count(int *sms);

@@ -1,0 +1,56 @@
+// merge_launch.cuh -- internal: launch templates of the merge / materialise
+// kernel, for one shared log length (NoSlots) or a list of slots with their
+// own lengths (SlotList).
+#pragma once
+
+#include "launch.h"
+
+namespace dl {
+namespace merge_detail {
+
+template <bool SLOTS>
+long long launch_heads(const MergeParams &p, const SlotArg<SLOTS> &sl) {
+    if constexpr (SLOTS)
+        return (long long)sl.n * p.H;
+    else
+        return p.NH;
+}
+
+// p.L is the shared length, or for a slot list the longest length in it.
+template <int OP, int DK, int DV, int TV, int LB, bool SLOTS>
+cudaError_t launch_lb(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
+    constexpr int NT = CtaShape<DK, TV>::NT;
+    static std::atomic<unsigned long long> smem_ok{0};
+    auto kern = merge_kernel<OP, DK, DV, TV, NT, LB, SLOTS>;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, true).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, true).bytes);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(launch_heads<SLOTS>(p, sl) * (DV / TV));
+    kern<<<grid, NT, smem, s>>>(p, sl);
+    return cudaGetLastError();
+}
+
+// The logged value factors stay in registers for logs of up to 8 entries.
+template <int OP, int DK, int DV, int TV, bool SLOTS>
+cudaError_t launch_tv(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
+    if (p.L <= 4) return launch_lb<OP, DK, DV, TV, 4, SLOTS>(p, sl, s);
+    if (p.L <= 8) return launch_lb<OP, DK, DV, TV, 8, SLOTS>(p, sl, s);
+    return launch_lb<OP, DK, DV, TV, 0, SLOTS>(p, sl, s);
+}
+
+template <int OP, int DK, int DV, bool SLOTS>
+cudaError_t launch(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    switch (pick_tile(launch_heads<SLOTS>(p, sl), DV, sms)) {
+        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, SLOTS>(p, sl, s); break;
+        case 64: return launch_tv<OP, DK, DV, 64, SLOTS>(p, sl, s);
+        default: break;
+    }
+    return launch_tv<OP, DK, DV, 32, SLOTS>(p, sl, s);
+}
+
+}  // namespace merge_detail
+}  // namespace dl

@@ -74,10 +74,22 @@ class DecodeLayer:
         shape = (self.w.heads, self.w.dv) if T is None else (T, self.w.heads, self.w.dv)
         return torch.empty(shape, dtype=self.out_dtype, device=self.device)
 
-    def step(self, x: dict, t: int, out: torch.Tensor, stream=None):
-        """Decode token t of the stacked inputs `x` into `out` [NH, dv]."""
+    def step(self, x: dict, t: int, out: torch.Tensor, stream=None, active=None):
+        """Decode token t of the stacked inputs `x` into `out` [NH, dv]; with
+        `active` (B truth values) only those slots decode."""
         beta = None if self.w.op == RWKV6 else x["beta"][t]
-        self.handle.decode_step(x["q"][t], x["k"][t], x["v"][t], beta, x["g"][t], out, stream)
+        self.handle.decode_step(x["q"][t], x["k"][t], x["v"][t], beta, x["g"][t], out, stream,
+                                active)
+
+    def slot_len(self, slot: int) -> int:
+        return self.handle.slot_len(slot)
+
+    def slot_reset(self, slot: int, S_new: torch.Tensor):
+        """Slot `slot` starts a new sequence from the dense state S_new
+        [H, dk, dv] (its log is dropped)."""
+        H = self.w.H
+        self.base[slot * H:(slot + 1) * H].copy_(S_new.reshape(H, self.w.dk, self.w.dv))
+        self.handle.slot_reset(slot)
 
     def materialize(self, stream=None) -> torch.Tensor:
         S = torch.empty_like(self.base)

@@ -189,13 +189,51 @@ def test_cycle_rejects_bad_layers(lib):
             with pytest.raises(B.DeltaLogError) as e:
                 B.dl_cycle_create(list(pair), io)
             assert e.value.status == B.DL_EINVAL
-        B.dl_decode_step(h1, None, None, None, None, None, None, stream=0)
-        with pytest.raises(B.DeltaLogError) as e:
-            B.dl_cycle_create([h1], [[(None,) * 6]] * 2)
-        assert e.value.status == B.DL_ESTATE
     finally:
         for h in (h1, h2, h3):
             B.dl_destroy(h)
+
+
+def test_slot_calls_check_arguments(lib):
+    hh = B.dl_create(cfg(B=3), 4096, 8192, None)
+    try:
+        for bad in (-1, 3):
+            with pytest.raises(B.DeltaLogError) as e:
+                B.dl_slot_reset(hh, bad)
+            assert e.value.status == B.DL_EINVAL
+            assert B.dl_slot_len(hh, bad) == -1
+        assert [B.dl_slot_len(hh, b) for b in range(3)] == [0, 0, 0]
+        B.dl_slot_reset(hh, 1)                      # already empty: nothing changes
+        assert B.dl_log_len(hh) == 0
+    finally:
+        B.dl_destroy(hh)
+    assert B.dl_slot_len(0, 0) == -1
+
+
+def test_idle_slots_launch_nothing(lib):
+    """A step in which no slot is active launches nothing and moves no length
+    (the fake device addresses are never touched)."""
+    hh = B.dl_create(cfg(B=3, C=2), 4096, 8192, None)
+    try:
+        a = 1 << 20
+        for _ in range(3):
+            B.dl_decode_step_masked(hh, [0, 0, 0], a, a, a, a, a, a, stream=0)
+        assert B.dl_log_len(hh) == 0
+    finally:
+        B.dl_destroy(hh)
+
+
+@pytest.mark.skipif(_has_gpu(), reason="checks the no-device failure path")
+def test_failed_slot_step_leaves_lengths(lib):
+    hh = B.dl_create(cfg(B=3, C=3), 4096, 8192, None)
+    try:
+        a = 1 << 20
+        with pytest.raises(B.DeltaLogError) as e:
+            B.dl_decode_step_masked(hh, [1, 0, 1], a, a, a, a, a, a, stream=0)
+        assert e.value.status == B.DL_ECUDA
+        assert [B.dl_slot_len(hh, b) for b in range(3)] == [0, 0, 0]
+    finally:
+        B.dl_destroy(hh)
 
 
 def test_strerror(lib):

@@ -378,3 +378,31 @@ def test_stack_largest_batch(C):
     layer), two of its layers, two cycles and a ragged third."""
     w = synth.WORKLOADS[f"gdn-stack24-b512-h16-d128-c{C}"]
     _full_size_check(w, layers=2, T=2 * C + 3)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("mode", MODES)
+def test_checkpoint_resume(op, mode):
+    """Checkpoint = materialise the logical state mid-cycle; resume = a new
+    handle over that dense state with an empty log.  The resumed run's
+    outputs and final state match the uninterrupted run's."""
+    C = 5
+    w = small(op, 128, 64, C=C, T=2 * C + 2, in_dt="bf16", out_dt="f32")
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    x = D.to_device(ti, w)
+    ref, outs_ref, _, _ = run_deltalog(w, x, S0, bonus, C, auto_merge=mode)
+    cut = C + 2                                   # mid-cycle: L = 2
+    first = D.DecodeLayer(w, S0, bonus, C=C, auto_merge=mode)
+    outs = first.new_out(w.T)
+    for t in range(cut):
+        first.step(x, t, outs[t])
+    assert first.L == 2
+    ckpt = first.materialize().cpu().numpy()
+    second = D.DecodeLayer(w, ckpt.reshape(w.B, w.H, w.dk, w.dv), bonus, C=C, auto_merge=mode)
+    for t in range(cut, w.T):
+        second.step(x, t, outs[t])
+    torch.cuda.synchronize()
+    assert rel_err(to_np(outs), to_np(outs_ref)) <= 1e-5
+    assert rel_err(to_np(second.materialize()), to_np(ref.materialize())) <= 1e-5
