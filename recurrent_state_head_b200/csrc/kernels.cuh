@@ -313,6 +313,41 @@ __device__ __forceinline__ void reduce_rows(float4 (&acc)[NA], float *red, float
     __syncthreads();
 }
 
+// The same partial sums, left with the threads below TV: thread c gets
+// column c's sums in xs[a] (the other threads' xs are not set).  One barrier
+// instead of two: the sums go straight to the value side.
+template <int NA, int TV, int NT>
+__device__ __forceinline__ void reduce_cols(float4 (&acc)[NA], float *red, float (&xs)[NA]) {
+    constexpr int TPR = TV / 4;
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int a = 0; a < NA; ++a) {
+#pragma unroll
+        for (int o = TPR; o < 32; o <<= 1) {
+            acc[a].x += __shfl_xor_sync(0xffffffffu, acc[a].x, o);
+            acc[a].y += __shfl_xor_sync(0xffffffffu, acc[a].y, o);
+            acc[a].z += __shfl_xor_sync(0xffffffffu, acc[a].z, o);
+            acc[a].w += __shfl_xor_sync(0xffffffffu, acc[a].w, o);
+        }
+    }
+    if (lane < TPR) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a)
+            *reinterpret_cast<float4 *>(&red[(a * NW + warp) * TV + lane * 4]) = acc[a];
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < TV) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) t += red[(a * NW + w) * TV + threadIdx.x];
+            xs[a] = t;
+        }
+    }
+}
+
 // ===================================================== operand staging ==
 //
 // The append, merge-token and merge kernels hold their base tile in
@@ -540,7 +575,6 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
     __shared__ __align__(16) float s_red[NA * T::NW * TV];
-    __shared__ float s_x[NA * TV];
     __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
     const int tid = threadIdx.x;
@@ -645,6 +679,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
     __syncthreads();
 
     // 4. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
+    float xc[NA];
     {
         float4 acc[NA];
 #pragma unroll
@@ -658,7 +693,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
                 fma4(acc[a], w, s[r]);
             }
         }
-        reduce_rows<NA, TV, NT>(acc, s_red, s_x);
+        reduce_cols<NA, TV, NT>(acc, s_red, xc);
     }
 
     // 5. value side: log replay, delta correction, output, append of u
@@ -671,7 +706,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             float rr = 0.f;
             for (int j = 0; j < L; ++j)
                 rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
-            const float o = p.scale * (s_x[c] + rr + s_self * vv);
+            const float o = p.scale * (xc[0] + rr + s_self * vv);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = vv;
@@ -686,8 +721,8 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
                 rq = fmaf(s_coef[1][j], uj, rq);
             }
             const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
-            const float u = beta * (vv - s_x[c] - rk);
-            const float o = p.scale * (s_x[TV + c] + rq + s_self * u);
+            const float u = beta * (vv - xc[0] - rk);
+            const float o = p.scale * (xc[NA - 1] + rq + s_self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
             if (FOLD)
                 s_u[c] = u;
