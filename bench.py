@@ -232,7 +232,7 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99):
     S_all = synth.initial_state(w).reshape(w.heads, w.dk, w.dv)
     bon_all = synth.bonus(w)
 
-    def run(n_heads, n_cycles):
+    def run(n_heads, n_cycles, n_threads=threads, eager=False):
         heads = np.sort(rng.choice(w.heads, size=min(n_heads, w.heads), replace=False))
         T = n_cycles * w.C
         ti = synth.tokens(w, 0, T, heads=heads)
@@ -240,11 +240,15 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99):
         if g.ndim == 2:
             g = g[:, :, None]
         bon = None if bon_all is None else bon_all[heads % w.H]
-        st = oracle.LogState(w.op, S_all[heads], w.C)
+        beta = None if w.op == 2 else ti.beta.astype(np.float64)
         t0 = time.perf_counter()
-        oracle.deltalog_run(st, ti.q64, ti.k64, ti.v64,
-                            None if w.op == 2 else ti.beta.astype(np.float64), g, bon,
-                            w.scale, n_threads=threads)
+        if eager:
+            oracle.eager_run(w.op, S_all[heads], ti.q64, ti.k64, ti.v64, beta, g, bon, w.scale,
+                             n_threads=n_threads)
+        else:
+            st = oracle.LogState(w.op, S_all[heads], w.C)
+            oracle.deltalog_run(st, ti.q64, ti.k64, ti.v64, beta, g, bon, w.scale,
+                                n_threads=n_threads)
         return time.perf_counter() - t0, len(heads), T
 
     probe = min(w.heads, max(4 * threads, 16))
@@ -254,9 +258,17 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99):
     n_heads = int(min(w.heads, max(probe, budget / w.C)))
     n_cycles = int(max(1, min(w.T // w.C, budget / (n_heads * w.C))))
     dt, n, T = run(n_heads, n_cycles)
+    # one thread, and the eager recurrence on all threads, on smaller samples
+    h1 = max(1, min(n_heads, int(0.15 * target_s / max(per_head_token * threads * w.C, 1e-9))))
+    dt1, n1, T1 = run(h1, 1, n_threads=1)
+    dte, ne, Te = run(n_heads, 1, eager=True)
     return {"value": n * T / dt / w.H, "unit": "tok/s", "cores": threads, "kind": "oracle",
             "sample": f"{n} of {w.heads} heads x {T} tokens ({n_cycles} merge cycles), "
-                      f"fp64 base+log oracle, {dt:.1f} s on {threads} threads"}
+                      f"fp64 base+log oracle, {dt:.1f} s on {threads} threads",
+            "value_1thread": n1 * T1 / dt1 / w.H,
+            "eager_value": ne * Te / dte / w.H,
+            "extra_samples": f"1 thread: {n1} heads x {T1} tokens in {dt1:.1f} s; eager: {ne} heads "
+                             f"x {Te} tokens in {dte:.1f} s on {threads} threads"}
 
 
 # ------------------------------------------------------------ native ----
