@@ -97,8 +97,8 @@ typedef struct dl_handle dl_handle;   /* opaque; host memory only */
  *                                  in_dtype copies of v (RWKV6)
  *   Lambda float [NH, C, m]        cumulative log-decay since the last merge,
  *                                  m = 1 (GDN) or d_k (KDA, RWKV6)
- * The log is the paper's "bounded update log" (gist.science technical
- * summary, "Meccanismo Core: Base + Log"). */
+ * The log is the paper's bounded log of compact update factors
+ * (gist.science technical summary, "Meccanismo Core: Base + Log"). */
 size_t dl_log_bytes(const dl_config *cfg);
 
 /* Byte offsets of the K, U and Lambda regions inside the log workspace. */
@@ -159,7 +159,7 @@ int dl_log_len(const dl_handle *h);
 /* Continuous batching: every slot b (batch row, heads b*H .. b*H + H-1)
  * keeps its own log length L_b, so sequences can join, leave and idle
  * independently and each slot merges when its own log is full.  The log of
- * a (slot, head) pair is the paper's per-"slot-head" unit (gist.science
+ * a (slot, head) pair is the paper's per-slot-head unit (gist.science
  * technical summary, "Implementazione del Kernel": ReplayPrep coefficients
  * are computed once per slot-head).  All slots start at L_b = 0; while every
  * slot has the same length and every slot decodes, nothing differs from
@@ -194,9 +194,9 @@ int dl_slot_len(const dl_handle *h, int slot);
 void dl_destroy(dl_handle *h);
 
 /* ------------------------------------------------------- merge cycle ---- */
-/* One merge cycle of several layers as a single CUDA graph (paper: split-
- * replay ablation "with CUDA Graph replay", latencies amortised over one
- * merge cycle, signal-papers page Fig. 9 caption).  The graph holds, token
+/* One merge cycle of several layers as a single CUDA graph (paper: the
+ * split-replay ablation replays its kernels from a CUDA graph and amortises
+ * latencies over one merge cycle, signal-papers page Fig. 9 caption).  The graph holds, token
  * by token, every layer's step; the C-th token of a layer is its
  * merge-token (DL_MERGE_FOLD: n_layers * C kernels) or its append followed
  * by its merge (DL_MERGE_SEPARATE: n_layers * (C + 1) kernels).
