@@ -63,7 +63,6 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
     cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
     switch (pick_tile(p.NH, DV, sms)) {
-        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, FOLD>(p, s); break;
         case 64: return launch_tv<OP, DK, DV, 64, FOLD>(p, s);
         default: break;
     }
@@ -90,7 +89,6 @@ cudaError_t launch_slots(const AppendParams &p, const SlotList &sl, cudaStream_t
     cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
     switch (pick_tile((long long)sl.n * p.H, DV, sms)) {
-        case 128: if constexpr (DV >= 128) return launch_slots_tv<OP, DK, DV, 128>(p, sl, s); break;
         case 64: return launch_slots_tv<OP, DK, DV, 64>(p, sl, s);
         default: break;
     }

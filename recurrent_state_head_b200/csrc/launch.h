@@ -31,10 +31,10 @@ merge_slots_fn get_merge_slots(int op, int dk, int dv);
 cudaError_t sm_count(int *sms);
 
 // Value-tile width for NH heads of width DV: 64 columns (or the whole head
-// when narrower) while that still gives at least four CTAs per SM, else the
-// widest tile that does (>= 32 columns).  Measured on B200 for d = 64 and 128:
-// 64-column tiles beat 32 (more per-CTA work to amortise the prologue) and
-// 128 (fewer, longer CTAs: worse overlap of their serial phases).
+// when narrower) while that still gives at least four CTAs per SM, else 32.
+// Measured on B200 for d = 64 and 128: 64-column tiles beat 32 (more per-CTA
+// work to amortise the prologue) and 128 (fewer, longer CTAs: worse overlap
+// of their serial phases), so 128-column tiles are not built.
 inline int pick_tile(long long NH, int DV, int sms) {
     int tv = DV < 64 ? DV : 64;
     while (tv > 32 && NH * (DV / tv) < 4LL * sms) tv /= 2;

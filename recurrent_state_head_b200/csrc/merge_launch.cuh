@@ -45,7 +45,6 @@ cudaError_t launch(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t 
     cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return e;
     switch (pick_tile(launch_heads<SLOTS>(p, sl), DV, sms)) {
-        case 128: if constexpr (DV >= 128) return launch_tv<OP, DK, DV, 128, SLOTS>(p, sl, s); break;
         case 64: return launch_tv<OP, DK, DV, 64, SLOTS>(p, sl, s);
         default: break;
     }
