@@ -47,6 +47,8 @@ struct AppendParams {
                               // previous kernel (launch is a programmatic
                               // dependent and the previous kernel does not
                               // write this base)
+    int stagger_ns, sms;      // append: the first wave's CTAs start
+                              // ((blockIdx / sms) mod 4) * stagger_ns apart
 };
 
 struct MergeParams {
@@ -598,6 +600,11 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             s[r] = FOLD ? ld_state_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first)
                         : ld_stream_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first);
     };
+    // The first wave's CTAs of an SM would otherwise run their serial phases
+    // in step, with none of them loading meanwhile; starting them a fraction
+    // of a CTA's lifetime apart keeps part of the SM streaming throughout.
+    if (!FOLD && p.stagger_ns > 0 && (int)blockIdx.x < 4 * p.sms)
+        __nanosleep((unsigned)(((int)blockIdx.x / p.sms) & 3) * (unsigned)p.stagger_ns);
     if (p.early) load_base();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
