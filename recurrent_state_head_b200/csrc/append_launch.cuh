@@ -9,11 +9,13 @@
 namespace dl {
 namespace append_detail {
 
-// Start offset between the first wave's CTAs of an SM (append only).
-// Measured on B200 in four-layer merge cycles against no offset: GDN -2.3 %,
-// KDA -1.2 %, RWKV6 -2.5 % per token at 1.0 us (0.6 us: the same for GDN
-// and KDA, -1 % for RWKV6; 1.5 us no better).
-constexpr int kStaggerNs = 1000;
+// The first wave's CTAs of an SM start spread over kStaggerWindowNs (slot i
+// of n resident CTAs at i * window / n).  Measured on B200 in four-layer
+// merge cycles, append with four CTAs per SM, against no offset: GDN -2.3 %,
+// KDA -1.2 %, RWKV6 -2.5 % per token with 1.0 us between CTAs (0.6 us: the
+// same for GDN and KDA, -1 % for RWKV6; 1.5 us no better).
+constexpr int kStaggerWindowNs = 4000;
+constexpr bool kStaggerFold = true;
 
 // Plain launch, or a programmatic dependent launch when p.early (it may
 // start while the previous kernel of the stream finishes; the kernel orders
@@ -48,13 +50,22 @@ cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((long long)p.NH * (DV / TV));
-    AppendParams q = p;
-    if constexpr (!FOLD) {
-        q.stagger_ns = kStaggerNs;
-        e = sm_count(&q.sms);
+    Stagger st{0, 0, 0};
+    if (!FOLD || kStaggerFold) {
+        static std::atomic<int> resident{0};
+        int slots = resident.load(std::memory_order_relaxed);
+        if (slots == 0) {
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&slots, kern, NT, smem);
+            if (e != cudaSuccess) return e;
+            slots = slots > 0 ? slots : 1;
+            resident.store(slots, std::memory_order_relaxed);
+        }
+        e = sm_count(&st.sms);
         if (e != cudaSuccess) return e;
+        st.slots = slots;
+        st.ns = kStaggerWindowNs / slots;
     }
-    return launch_kernel(kern, grid, NT, smem, q.early != 0, s, q);
+    return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p, st);
 }
 
 // The merge-token keeps the logged value factors in registers while the log

@@ -172,8 +172,6 @@ dl::AppendParams append_params(const dl_handle *h, const dl_step_io &io, int L) 
     p.in_bf16 = h->cfg.in_dtype == DL_BF16;
     p.out_bf16 = h->cfg.out_dtype == DL_BF16;
     p.early = 0;
-    p.stagger_ns = 0;
-    p.sms = 0;
     return p;
 }
 

@@ -47,8 +47,12 @@ struct AppendParams {
                               // previous kernel (launch is a programmatic
                               // dependent and the previous kernel does not
                               // write this base)
-    int stagger_ns, sms;      // append: the first wave's CTAs start
-                              // ((blockIdx / sms) mod 4) * stagger_ns apart
+};
+
+// Start offsets of the first wave's CTAs: CTA b < slots * sms starts
+// (b / sms) * ns nanoseconds late (slots = CTAs resident per SM).
+struct Stagger {
+    int ns, slots, sms;
 };
 
 struct MergeParams {
@@ -600,11 +604,6 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             s[r] = FOLD ? ld_state_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first)
                         : ld_stream_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first);
     };
-    // The first wave's CTAs of an SM would otherwise run their serial phases
-    // in step, with none of them loading meanwhile; starting them a fraction
-    // of a CTA's lifetime apart keeps part of the SM streaming throughout.
-    if (!FOLD && p.stagger_ns > 0 && (int)blockIdx.x < 4 * p.sms)
-        __nanosleep((unsigned)(((int)blockIdx.x / p.sms) & 3) * (unsigned)p.stagger_ns);
     if (p.early) load_base();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -772,8 +771,13 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
 
 template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0>
 __global__ void __launch_bounds__(NT)
-append_kernel(const AppendParams p) {
+append_kernel(const AppendParams p, const Stagger st) {
     using T = Tile<DK, DV, TV, NT>;
+    // The first wave's CTAs of an SM would otherwise run their serial phases
+    // in step, with none of them loading meanwhile; starting them a fraction
+    // of a CTA's lifetime apart keeps part of the SM streaming throughout.
+    if (st.ns > 0 && (int)blockIdx.x < st.slots * st.sms)
+        __nanosleep((unsigned)((int)blockIdx.x / st.sms) * (unsigned)st.ns);
     const int lh = (int)blockIdx.x / T::NVT;
     append_unit<OP, DK, DV, TV, NT, FOLD, LB>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
 }
