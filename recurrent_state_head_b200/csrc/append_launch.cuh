@@ -42,7 +42,7 @@ cudaError_t launch_kernel(Kernel kern, unsigned grid, int threads, size_t smem, 
 
 template <int OP, int DK, int DV, int TV, bool FOLD, int LB>
 cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
-    constexpr int NT = CtaShape<DK, TV>::NT;
+    constexpr int NT = AppendShape<DK, TV, FOLD>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB>;
     const int ie = p.in_bf16 ? 2 : 4;
