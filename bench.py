@@ -200,15 +200,25 @@ def measured_peaks():
         return dict(PEAKS_FALLBACK)
 
 
+def kernel_source_digest(path):
+    """sha256 of a CUDA source with its comments and blank space removed, so
+    that it changes exactly when the code does."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()
+
+
 def recorded_traffic(workload_name):
     """Per-launch DRAM bytes of the append kernel from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
+    summary, if it was taken on the current kernel code (else None)."""
     path = os.path.join(ROOT, "profiles", f"append_kernel_{workload_name}.md")
     src = os.path.join(ROOT, "recurrent_state_head_b200", "csrc", "kernels.cuh")
     try:
         text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+        sha = kernel_source_digest(src)
+        m_sha = re.search(r"kernel_code_sha256:\s*([0-9a-f]{64})", text)
         m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
         if m_sha and m_b and m_sha.group(1) == sha:
             return float(m_b.group(1))
