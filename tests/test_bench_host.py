@@ -1,0 +1,49 @@
+"""Host-side pieces of bench.py that need no GPU: the key that ties the
+recorded ncu traffic to the kernel code, and the byte model's write
+reduction on every workload (the C/2 bar of the measurement)."""
+import os
+
+import pytest
+
+import bench
+from recurrent_state_head_b200 import synth
+
+CODE = """// a comment
+__device__ float f(float x) {   /* block
+   comment */ return x * 2.f; }
+"""
+
+
+def test_code_digest_ignores_comments_and_blank_space(tmp_path):
+    a, b, c = tmp_path / "a.cuh", tmp_path / "b.cuh", tmp_path / "c.cuh"
+    a.write_text(CODE)
+    b.write_text(CODE.replace("// a comment", "// another comment\n\n").replace("   ", " "))
+    c.write_text(CODE.replace("2.f", "3.f"))
+    assert bench.kernel_source_digest(str(a)) == bench.kernel_source_digest(str(b))
+    assert bench.kernel_source_digest(str(a)) != bench.kernel_source_digest(str(c))
+
+
+def test_recorded_traffic_matches_the_committed_profile():
+    """The committed append summary was taken on the current kernel code, so
+    the bench reports its traffic; it is within a few percent of the
+    algorithmic bytes of one launch at the cycle's mean log length."""
+    w = synth.WORKLOADS["gdn-b128-h16-d128-c8"]
+    t = bench.recorded_traffic(w.name)
+    assert t is not None
+    bm = bench.bytes_model(w)
+    algo = w.heads * sum(bm["append"](3))
+    assert 0.95 < t / algo < 1.1
+
+
+def test_recorded_traffic_absent_for_unprofiled_workload():
+    assert bench.recorded_traffic("no-such-workload") is None
+
+
+@pytest.mark.parametrize("name", [n for n in synth.WORKLOADS if "stack24" not in n or "b128" in n])
+def test_write_reduction_meets_half_capacity(name):
+    w = synth.WORKLOADS[name]
+    bm = bench.bytes_model(w)
+    ratio = bm["eager"][1] / bm["token_write"]
+    assert ratio >= w.C / 2, (name, ratio)
+    # the merge-token never writes more than the separate merge
+    assert bm["token_write"] <= bench.bytes_model(w, fold=False)["token_write"]
