@@ -175,7 +175,8 @@ int dl_log_len(const dl_handle *h);
  * and one merge kernel (DL_MERGE_SEPARATE: the slots that reach C), each
  * over just its slots (split into launches of at most 512 slots).
  * Errors: as dl_decode_step; DL_ESTATE if an active slot's log is full
- * with DL_MERGE_OFF (nothing launched, no length moves). */
+ * with DL_MERGE_OFF (nothing launched, no length moves); DL_EINVAL if the
+ * step needs per-slot lengths and B > 65536 (slot lists carry 16-bit ids). */
 dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const void *q,
                                 const void *k, const void *v, const float *beta,
                                 const float *g, void *out, void *stream);
@@ -184,7 +185,8 @@ dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const
  * dropped.  The slot's base rows ([H, d_k, d_v] at head slot*H) are the
  * caller's to fill with the sequence's starting state (zeros, or the state
  * a prefill produced) before the next call that reads them.  Host-side
- * only: nothing is launched.  Errors: DL_EINVAL (NULL handle, bad slot). */
+ * only: nothing is launched.  Errors: DL_EINVAL (NULL handle, bad slot, or
+ * B > 65536 while the slot's log is not empty). */
 dl_status dl_slot_reset(dl_handle *h, int slot);
 
 /* Log length of one slot, or -1 for a NULL handle or a slot out of range. */

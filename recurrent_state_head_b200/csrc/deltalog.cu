@@ -97,6 +97,9 @@ dl_status check_step_ptrs(const dl_config *c, const void *q, const void *k, cons
 
 namespace {
 
+// Slot ids travel to the kernels as 16-bit list entries.
+constexpr int kMaxSlotId = 65535;
+
 // Log lengths of a handle's slots: one shared length while every slot has
 // it (the common case), else one length per slot.
 struct Lens {
@@ -293,6 +296,8 @@ dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active,
     // active slots, merge-token slots (DL_MERGE_FOLD, log one short of full)
     // first; with DL_MERGE_SEPARATE the slots that fill their log are then
     // merged by the merge kernel
+    if (B > kMaxSlotId + 1)
+        return fail(DL_EINVAL, "per-slot lengths support at most %d slots (B = %d)", kMaxSlotId + 1, B);
     std::vector<int> ids, lens, idm, lm;
     int nfold = 0;
     for (int pass = 0; pass < 2; ++pass)
@@ -475,6 +480,8 @@ dl_status dl_slot_reset(dl_handle *h, int slot) {
     if (!h) return fail(DL_EINVAL, "handle is NULL");
     if (slot < 0 || slot >= h->cfg.B) return fail(DL_EINVAL, "slot %d outside [0, %d)", slot, h->cfg.B);
     if (h->lens.of(slot) == 0) return ok();
+    if (h->cfg.B > kMaxSlotId + 1)
+        return fail(DL_EINVAL, "per-slot lengths support at most %d slots (B = %d)", kMaxSlotId + 1, h->cfg.B);
     h->lens.split(h->cfg.B);
     h->lens.per[(size_t)slot] = 0;
     h->lens.join();

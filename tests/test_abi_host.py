@@ -236,6 +236,20 @@ def test_failed_slot_step_leaves_lengths(lib):
         B.dl_destroy(hh)
 
 
+def test_per_slot_lengths_need_16_bit_slot_ids(lib):
+    """Slot lists carry 16-bit ids: with more slots, steps that need per-slot
+    lengths are refused before any launch (shared-length steps still run)."""
+    hh = B.dl_create(cfg(B=70000, H=1), 4096, 8192, None)
+    try:
+        a = 1 << 20
+        with pytest.raises(B.DeltaLogError) as e:
+            B.dl_decode_step_masked(hh, [1] + [0] * 69999, a, a, a, a, a, a, stream=0)
+        assert e.value.status == B.DL_EINVAL
+        assert B.dl_log_len(hh) == 0
+    finally:
+        B.dl_destroy(hh)
+
+
 def test_strerror(lib):
     for s in range(5):
         assert B.dl_strerror(s)
