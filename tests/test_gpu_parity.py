@@ -406,3 +406,29 @@ def test_checkpoint_resume(op, mode):
     torch.cuda.synchronize()
     assert rel_err(to_np(outs), to_np(outs_ref)) <= 1e-5
     assert rel_err(to_np(second.materialize()), to_np(ref.materialize())) <= 1e-5
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("mode", MODES)
+def test_strong_decay_long_log(op, mode):
+    """C = 16 with log-decays eight times the usual scale (the cumulative
+    decay over a cycle reaches e^-100): outputs and states against the
+    eager oracle, no overflow or NaN in the replay factors."""
+    C = 16
+    w = small(op, 128, 64, C=C, T=2 * C + 5, in_dt="bf16", out_dt="f32", seed=91)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, w.T)
+    ti.g[...] = (ti.g.astype(np.float64) * 8.0).astype(np.float32)
+    x = D.to_device(ti, w)
+    layer, outs, Ls, mats = run_deltalog(w, x, S0, bonus, C, check_every_step=True,
+                                         auto_merge=mode)
+    Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, S0=S0, bonus=bonus)
+    S = Sr
+    o = to_np(outs)
+    assert np.all(np.isfinite(o))
+    for t in range(w.T):
+        S, o_ref = run_oracle_eager(w, S, q[t:t + 1], k[t:t + 1], v[t:t + 1], beta[t:t + 1],
+                                    g[t:t + 1], bon)
+        assert rel_err(o[t], o_ref[0]) <= tol_out(w), t
+        assert rel_err(mats[t], S) <= TOL_STATE, t

@@ -256,6 +256,26 @@ def test_base_log_matches_eager_bruteforce(oracle_lib, op, dims):
 
 
 @pytest.mark.parametrize("op", OPS)
+def test_base_log_with_strong_decay_over_a_long_log(oracle_lib, op):
+    """C = 16 with log-decays eight times the usual scale: the cumulative
+    decay over a cycle reaches e^-100 and below.  The replay factors
+    e^(Lambda_t - Lambda_j) stay bounded by 1, so the base + log formulation
+    still equals the eager recurrence (a formulation that divided the keys
+    by the decay would overflow here)."""
+    rng = np.random.default_rng(41 + op)
+    nh, dk, dv, C, T = 2, 4, 3, 16, 40
+    S0 = rng.standard_normal((nh, dk, dv))
+    q, k, v, beta, g, bonus = rand_inputs(rng, op, nh, dk, dv, T, g_scale=8.0)
+    b_ = None if op == RWKV6 else beta
+    S_e, o_e = oracle.eager_run(op, S0, q, k, v, b_, g, bonus, 0.5)
+    st = LogState(op, S0, C)
+    o_l, _, _ = oracle.deltalog_run(st, q, k, v, b_, g, bonus, 0.5)
+    assert np.all(np.isfinite(o_l)) and np.all(np.isfinite(st.base))
+    assert rel_err(o_l, o_e) < 1e-11
+    assert rel_err(oracle.materialize(st), S_e) < 1e-11
+
+
+@pytest.mark.parametrize("op", OPS)
 def test_capacity_one_is_eager(oracle_lib, op):
     rng = np.random.default_rng(9)
     nh, dk, dv, T = 3, 8, 5, 20
