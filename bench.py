@@ -229,7 +229,7 @@ def recorded_traffic(workload_name):
 
 # ------------------------------------------------------- CPU oracle -----
 
-def cpu_oracle_sample(w, target_s=12.0, seed=99):
+def cpu_oracle_sample(w, target_s=12.0, seed=99, extras=True):
     """Time the fp64 oracle's base+log decode on a bounded sample of the
     workload -- a random subset of its heads over whole merge cycles -- sized
     to about `target_s` seconds of host work.  Returns tok/s in the GPU's
@@ -268,17 +268,20 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99):
     n_heads = int(min(w.heads, max(probe, budget / w.C)))
     n_cycles = int(max(1, min(w.T // w.C, budget / (n_heads * w.C))))
     dt, n, T = run(n_heads, n_cycles)
+    out = {"value": n * T / dt / w.H, "unit": "tok/s", "cores": threads, "kind": "oracle",
+           "sample": f"{n} of {w.heads} heads x {T} tokens ({n_cycles} merge cycles), "
+                     f"fp64 base+log oracle, {dt:.1f} s on {threads} threads"}
+    if not extras:
+        return out
     # one thread, and the eager recurrence on all threads, on smaller samples
     h1 = max(1, min(n_heads, int(0.15 * target_s / max(per_head_token * threads * w.C, 1e-9))))
     dt1, n1, T1 = run(h1, 1, n_threads=1)
     dte, ne, Te = run(n_heads, 1, eager=True)
-    return {"value": n * T / dt / w.H, "unit": "tok/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {w.heads} heads x {T} tokens ({n_cycles} merge cycles), "
-                      f"fp64 base+log oracle, {dt:.1f} s on {threads} threads",
-            "value_1thread": n1 * T1 / dt1 / w.H,
-            "eager_value": ne * Te / dte / w.H,
-            "extra_samples": f"1 thread: {n1} heads x {T1} tokens in {dt1:.1f} s; eager: {ne} heads "
-                             f"x {Te} tokens in {dte:.1f} s on {threads} threads"}
+    out.update({"value_1thread": n1 * T1 / dt1 / w.H,
+                "eager_value": ne * Te / dte / w.H,
+                "extra_samples": f"1 thread: {n1} heads x {T1} tokens in {dt1:.1f} s; eager: {ne} heads "
+                                 f"x {Te} tokens in {dte:.1f} s on {threads} threads"})
+    return out
 
 
 # ------------------------------------------------------------ native ----
@@ -577,11 +580,11 @@ def run_reference(args, rank, world):
     w = synth.WORKLOADS[args.workload]
     per_step_s = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, target_s=per_step_s)
+        cpu_oracle_sample(w, target_s=per_step_s, extras=False)
     vals, samples = [], []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = cpu_oracle_sample(w, target_s=per_step_s)
+        r = cpu_oracle_sample(w, target_s=per_step_s, extras=False)
         vals.append(r["value"])
         samples.append(r)
     wall = time.perf_counter() - t0
