@@ -109,8 +109,15 @@ dl_status dl_log_layout(const dl_config *cfg, size_t *off_K, size_t *off_U,
  * [NH, d_k, d_v], 16-byte aligned, holds S at the last merge) and log
  * workspace (device, dl_log_bytes(cfg) bytes, 16-byte aligned).  `bonus` is
  * the RWKV6 bonus [H, d_k] (device, float, 16-byte aligned; ignored for the
- * other operators).  The
- * log starts empty (L = 0); its contents are never read before written.
+ * other operators).  The pair (base, log) is the paper's representation of
+ * the recurrent state: a dense base holding the history up to the last merge
+ * and a bounded buffer of compact update factors with their log-decay
+ * metadata (gist.science technical summary, "Meccanismo Core: Base + Log";
+ * signal-papers page, Fig. 4 caption).  The log starts empty (L = 0), as
+ * right after a merge; its contents are never read before written.  Any
+ * dense state can serve as the base, e.g. one a prefill produced.
+ * Host-side only: nothing is launched or allocated on the device; the handle
+ * (host memory) belongs to the caller until dl_destroy.
  * Errors: DL_EINVAL (config, NULL or misaligned pointer), DL_ENOMEM. */
 dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,
                     const float *bonus, dl_handle **out);
@@ -124,22 +131,30 @@ dl_status dl_create(const dl_config *cfg, float *base, void *log_ws,
  * this token included, is written over the base by the same kernel), with
  * DL_MERGE_SEPARATE the merge kernel runs after its append; either way L
  * returns to 0.
- * Errors: DL_EINVAL (NULL / misaligned pointer), DL_ESTATE (log full with
- * DL_MERGE_OFF; nothing launched), DL_ECUDA (launch failed; L unchanged if
- * the first kernel failed, L = C if only the separate merge failed). */
+ * Errors: DL_EINVAL (NULL / misaligned pointer; nothing launched),
+ * DL_ESTATE (L = C: the log is full with DL_MERGE_OFF, or a separate merge
+ * failed to launch earlier; nothing launched -- call dl_merge), DL_ECUDA (a
+ * launch failed: L is unchanged if the append or merge-token kernel did not
+ * launch; L = C if the append launched but the separate merge did not). */
 dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
                          const float *beta, const float *g, void *out, void *stream);
 
-/* Merge phase (paper: "Fase di Merge"): Sbar <- D(exp(Lambda_L)) Sbar +
+/* Merge phase (paper: "Fase di Merge", gist.science technical summary;
+ * signal-papers page, Fig. 4 caption): Sbar <- D(exp(Lambda_L)) Sbar +
  * sum_j D(exp(Lambda_L - Lambda_j)) k_j u_j^T in place, then L = 0 (every
  * slot at its own length L_b; slots at 0 are left as they are).
- * A no-op when L = 0.  Errors: DL_ECUDA. */
+ * A no-op when L = 0.  Errors: DL_ECUDA (the slots whose merge launched are
+ * at 0, the others keep their lengths). */
 dl_status dl_merge(dl_handle *h, void *stream);
 
 /* Write the logical state (base + replayed log) to S_out (device fp32
  * [NH, d_k, d_v], 16-byte aligned, must not overlap the base); base and log
- * are left untouched.  With L = 0 this copies the base.
- * Errors: DL_EINVAL, DL_ECUDA. */
+ * are left untouched.  With L = 0 this copies the base.  This is the
+ * merge's materialisation of the accumulated logical state (gist.science
+ * technical summary, "Fase di Merge") written out of place -- the state
+ * whose error the paper reports (signal-papers page, Fig. 12(b),
+ * materialized recurrent-state relative error); use it for checks and
+ * checkpoints.  Errors: DL_EINVAL, DL_ECUDA. */
 dl_status dl_materialize(const dl_handle *h, float *S_out, void *stream);
 
 /* Eager dense step (the in-house dense baseline; paper: eager decoding that
@@ -152,7 +167,10 @@ dl_status dl_eager_step(const dl_config *cfg, float *S, const void *q, const voi
                         const float *bonus, void *out, void *stream);
 
 /* The log length L (0 <= L <= C) every slot has, -2 when the slots'
- * lengths differ (see dl_slot_len), or -1 for a NULL handle. */
+ * lengths differ (see dl_slot_len), or -1 for a NULL handle.  L is the
+ * count in the paper's schedule (signal-papers page, Fig. 4 caption: append
+ * while L < C, materialise into the base when L = C); with an automatic
+ * merge mode it is (tokens since the last merge) mod C between calls. */
 int dl_log_len(const dl_handle *h);
 
 /* --------------------------------------------- per-slot log lengths ---- */
@@ -175,8 +193,13 @@ int dl_log_len(const dl_handle *h);
  * and one merge kernel (DL_MERGE_SEPARATE: the slots that reach C), each
  * over just its slots (split into launches of at most 512 slots).
  * Errors: as dl_decode_step; DL_ESTATE if an active slot's log is full
- * with DL_MERGE_OFF (nothing launched, no length moves); DL_EINVAL if the
- * step needs per-slot lengths and B > 65536 (slot lists carry 16-bit ids). */
+ * (nothing launched, no length moves); DL_EINVAL if the step needs per-slot
+ * lengths and B > 65536 (slot lists carry 16-bit ids).  After DL_ECUDA each
+ * slot's length tells what happened to it: a slot whose kernel launched has
+ * taken the step (L_b + 1, or 0 after its merge-token; with
+ * DL_MERGE_SEPARATE L_b = C until its merge launched), the others kept
+ * their lengths.  Retrying the step for every slot would apply the token
+ * twice to the slots that took it: compare dl_slot_len before retrying. */
 dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const void *q,
                                 const void *k, const void *v, const float *beta,
                                 const float *g, void *out, void *stream);
@@ -192,7 +215,11 @@ dl_status dl_slot_reset(dl_handle *h, int slot);
 /* Log length of one slot, or -1 for a NULL handle or a slot out of range. */
 int dl_slot_len(const dl_handle *h, int slot);
 
-/* Release the handle (host memory only).  NULL is accepted. */
+/* Release the handle (host memory only).  NULL is accepted.  The base and
+ * log workspace -- the state of "Meccanismo Core: Base + Log" (gist.science
+ * technical summary) -- stay the caller's and are not touched; work already
+ * queued on a stream keeps using them.  The pages define no release call;
+ * this ends the host-side bookkeeping of that state. */
 void dl_destroy(dl_handle *h);
 
 /* ------------------------------------------------------- merge cycle ---- */
@@ -231,9 +258,23 @@ int dl_cycle_kernels(const dl_cycle *cy);
 void dl_cycle_destroy(dl_cycle *cy);
 
 /* ------------------------------------------------------------ errors ---- */
+/* Name of a status code.  The pages describe no API, so no passage defines
+ * the codes themselves; DL_ESTATE is the one state their schedule forbids
+ * (a step when the log already holds C entries, signal-papers page, Fig. 4
+ * caption).  Never NULL. */
 const char *dl_strerror(dl_status s);
 /* Detail of the last error on the calling thread ("" if none). */
 const char *dl_last_error(void);
+
+/* ---------------------------------------------------------- testing ---- */
+/* Failure injection for tests of the log-length bookkeeping on machines
+ * with or without a GPU (no passage of the paper corresponds: this checks
+ * the error semantics above).  n_ok >= 0: from now on no kernel is issued
+ * at all -- the next n_ok launches are reported as launched (nothing is
+ * computed, no memory is touched) and every later one as failed
+ * (DL_ECUDA).  n_ok < 0 (the initial state): launches are issued normally.
+ * Process-wide; not for use outside tests. */
+void dl_debug_fake_launches(long long n_ok);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,7 @@ EXPORTS = (
     "dl_materialize", "dl_eager_step", "dl_log_len", "dl_destroy",
     "dl_decode_step_masked", "dl_slot_reset", "dl_slot_len",
     "dl_cycle_create", "dl_cycle_launch", "dl_cycle_kernels", "dl_cycle_destroy",
-    "dl_strerror", "dl_last_error",
+    "dl_strerror", "dl_last_error", "dl_debug_fake_launches",
 )
 
 
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.dl_cycle_destroy.argtypes, L.dl_cycle_destroy.restype = [P], None
             L.dl_strerror.argtypes, L.dl_strerror.restype = [I], ctypes.c_char_p
             L.dl_last_error.argtypes, L.dl_last_error.restype = [], ctypes.c_char_p
+            L.dl_debug_fake_launches.argtypes = [ctypes.c_longlong]
+            L.dl_debug_fake_launches.restype = None
             for f in ("dl_log_layout", "dl_create", "dl_decode_step", "dl_merge",
                       "dl_materialize", "dl_eager_step", "dl_cycle_create",
                       "dl_cycle_launch"):
@@ -220,6 +222,12 @@ def dl_strerror(status: int) -> str:
 
 def dl_last_error() -> str:
     return lib().dl_last_error().decode()
+
+
+def dl_debug_fake_launches(n_ok: int):
+    """Test hook: with n_ok >= 0 no kernel is issued; the next n_ok launches
+    report success, later ones fail.  n_ok < 0 restores real launches."""
+    lib().dl_debug_fake_launches(int(n_ok))
 
 
 # ------------------------------------------------------------- owners ----

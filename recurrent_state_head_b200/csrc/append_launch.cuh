@@ -44,22 +44,19 @@ template <int OP, int DK, int DV, int TV, bool FOLD, int LB>
 cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = AppendShape<DK, TV, FOLD>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
+    static std::atomic<int> resident[64];
     auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
-    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes);
+    const size_t smem_max = op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, smem_max);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((long long)p.NH * (DV / TV));
     Stagger st{0, 0, 0};
     if (!FOLD || kStaggerFold) {
-        static std::atomic<int> resident{0};
-        int slots = resident.load(std::memory_order_relaxed);
-        if (slots == 0) {
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&slots, kern, NT, smem);
-            if (e != cudaSuccess) return e;
-            slots = slots > 0 ? slots : 1;
-            resident.store(slots, std::memory_order_relaxed);
-        }
+        int slots = 1;
+        e = resident_ctas(resident, kern, NT, smem_max, &slots);
+        if (e != cudaSuccess) return e;
         e = sm_count(&st.sms);
         if (e != cudaSuccess) return e;
         st.slots = slots;

@@ -6,6 +6,7 @@
 // Attention Decoding" (arXiv 2608.15533): append / merge phases (gist.science
 // technical summary, "Meccanismo Core: Base + Log"; signal-papers page,
 // Fig. 4 caption) and CUDA-Graph replay of one merge cycle (Fig. 9 caption).
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -154,6 +155,22 @@ struct dl_cycle {
 
 namespace {
 
+// Failure injection for host tests of the length bookkeeping
+// (dl_debug_fake_launches): -1 issues every launch; n >= 0 issues none,
+// reports the next n as launched and every later one as failed.
+std::atomic<long long> g_fake_ok{-1};
+
+template <typename Launch>
+cudaError_t issue(Launch &&launch) {
+    long long left = g_fake_ok.load(std::memory_order_relaxed);
+    while (left >= 0) {
+        if (left == 0) return cudaErrorLaunchFailure;
+        if (g_fake_ok.compare_exchange_weak(left, left - 1, std::memory_order_relaxed))
+            return cudaSuccess;
+    }
+    return launch();
+}
+
 dl::AppendParams append_params(const dl_handle *h, const dl_step_io &io, int L) {
     dl::AppendParams p;
     p.base = h->base;
@@ -204,10 +221,11 @@ cudaError_t launch_append(const dl_handle *h, const dl_step_io &io, int L, bool 
     if (h->NH == 0) return cudaSuccess;
     dl::AppendParams p = append_params(h, io, L);
     p.early = early ? 1 : 0;
-    return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, fold, s);
+    return issue([&] { return dl::get_append(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, fold, s); });
 }
 
-// Do the layers' base states occupy pairwise disjoint memory?
+// Do the layers' base states occupy pairwise disjoint memory?  (Layers
+// without heads occupy none.)
 bool disjoint_bases(dl_handle *const *layers, int n) {
     for (int a = 0; a < n; ++a)
         for (int b = a + 1; b < n; ++b) {
@@ -222,17 +240,22 @@ bool disjoint_bases(dl_handle *const *layers, int n) {
 
 cudaError_t launch_merge(const dl_handle *h, float *dst, int L, cudaStream_t s) {
     if (h->NH == 0) return cudaSuccess;
-    return dl::get_merge(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, L), s);
+    return issue([&] { return dl::get_merge(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, L), s); });
 }
 
 // Slot-list launches of at most MAXSEL slots each: `ids` are the slots,
 // `lens` their lengths.  merge == false: the append kernel, whose first
 // `nfold` entries take the merge-token; merge == true: the merge kernel into
-// dst.
+// dst.  *done (if given) receives how many leading entries of `ids` were
+// launched, all of them on success.
 cudaError_t launch_slots(const dl_handle *h, bool merge, const std::vector<int> &ids,
                          const std::vector<int> &lens, int nfold, const dl_step_io *io, float *dst,
-                         cudaStream_t s, bool early, int *kernels) {
-    if (h->NH == 0) return cudaSuccess;
+                         cudaStream_t s, bool early, int *kernels, size_t *done = nullptr) {
+    if (done) *done = 0;
+    if (h->NH == 0) {
+        if (done) *done = ids.size();
+        return cudaSuccess;
+    }
     for (size_t at = 0; at < ids.size(); at += dl::MAXSEL) {
         const size_t n = ids.size() - at < (size_t)dl::MAXSEL ? ids.size() - at : (size_t)dl::MAXSEL;
         dl::SlotList sl;
@@ -247,30 +270,39 @@ cudaError_t launch_slots(const dl_handle *h, bool merge, const std::vector<int> 
         }
         cudaError_t e;
         if (merge) {
-            e = dl::get_merge_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, Lmax), sl, s);
+            e = issue([&] {
+                return dl::get_merge_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(merge_params(h, dst, Lmax), sl, s);
+            });
         } else {
             dl::AppendParams p = append_params(h, *io, Lmax);
             p.early = early ? 1 : 0;
-            e = dl::get_append_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, sl, s);
+            e = issue([&] { return dl::get_append_slots(h->cfg.op, h->cfg.dk, h->cfg.dv)(p, sl, s); });
         }
         if (e != cudaSuccess) return e;
         if (kernels) *kernels += 1;
+        if (done) *done = at + n;
     }
     return cudaSuccess;
 }
 
 // One decode token for the active slots (active == nullptr: all of them),
-// launched on `st`, with the lengths in `ln` (advanced on success).
-// Returns DL_OK, DL_ESTATE (nothing launched) or DL_ECUDA (lengths unchanged).
+// launched on `st`, with the lengths in `ln`.  Returns DL_OK, DL_ESTATE
+// (nothing launched, nothing moved) or DL_ECUDA.  Every length in `ln` is
+// kept true to what was launched: a slot whose kernel launched has taken
+// the step (L + 1, or 0 after its merge-token; with DL_MERGE_SEPARATE a
+// slot whose log filled stays at C until its merge launches), a slot whose
+// kernel did not launch keeps its length.
 dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active, const dl_step_io &io,
                       cudaStream_t st, bool early, int *kernels) {
     const int B = h->cfg.B, C = h->cfg.C, mode = h->cfg.auto_merge;
+    const char *full_msg = mode == DL_MERGE_OFF
+                               ? "log is full (L = C = %d) and auto_merge is off: merge first"
+                               : "log is full (L = C = %d) after a failed merge launch: call dl_merge";
     bool all = true;
     if (active)
         for (int b = 0; b < B && all; ++b) all = active[b] != 0;
     if (ln.shared && all) {
-        if (ln.L >= C)
-            return fail(DL_ESTATE, "log is full (L = C = %d) and auto_merge is off: merge first", C);
+        if (ln.L >= C) return fail(DL_ESTATE, full_msg, C);
         if (mode == DL_MERGE_FOLD && ln.L == C - 1) {
             // the token that completes the log: one kernel reads the base once
             // and writes the merged logical state back
@@ -286,7 +318,7 @@ dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active,
         ln.L += 1;
         if (mode == DL_MERGE_SEPARATE && ln.L == C) {
             e = launch_merge(h, h->base, ln.L, st);
-            if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
+            if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch (the log stays full)");
             if (kernels && h->NH > 0) *kernels += 1;
             ln.L = 0;
         }
@@ -304,9 +336,11 @@ dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active,
         for (int b = 0; b < B; ++b) {
             if (active && !active[b]) continue;
             const int L = ln.of(b);
-            if (L >= C)
-                return fail(DL_ESTATE, "slot %d's log is full (L = C = %d) and auto_merge is off: merge first",
-                            b, C);
+            if (L >= C) {
+                char msg[160];
+                snprintf(msg, sizeof msg, "slot %d: %s", b, full_msg);
+                return fail(DL_ESTATE, msg, C);
+            }
             const bool fold = mode == DL_MERGE_FOLD && L == C - 1;
             if (fold != (pass == 0)) continue;
             ids.push_back(b);
@@ -317,16 +351,19 @@ dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active,
                 lm.push_back(C);
             }
         }
-    cudaError_t e = launch_slots(h, false, ids, lens, nfold, &io, nullptr, st, early, kernels);
-    if (e == cudaSuccess) e = launch_slots(h, true, idm, lm, 0, nullptr, h->base, st, false, kernels);
-    if (e != cudaSuccess) return cuda_fail(e, "per-slot kernel launch");
+    if (ids.empty()) return ok();
+    size_t done = 0, merged = 0;
+    cudaError_t e = launch_slots(h, false, ids, lens, nfold, &io, nullptr, st, early, kernels, &done);
+    if (e == cudaSuccess) e = launch_slots(h, true, idm, lm, 0, nullptr, h->base, st, false, kernels, &merged);
     ln.split(B);
-    for (int b = 0; b < B; ++b) {
-        if (active && !active[b]) continue;
-        const int L = ln.per[(size_t)b] + 1;
-        ln.per[(size_t)b] = (unsigned char)((mode != DL_MERGE_OFF && L == C) ? 0 : L);
+    for (size_t i = 0; i < done; ++i) {
+        const size_t b = (size_t)ids[i];
+        const int L = ln.per[b] + 1;
+        ln.per[b] = (unsigned char)((mode == DL_MERGE_FOLD && L == C) ? 0 : L);
     }
+    for (size_t i = 0; i < merged; ++i) ln.per[(size_t)idm[i]] = 0;
     ln.join();
+    if (e != cudaSuccess) return cuda_fail(e, "per-slot kernel launch");
     return ok();
 }
 
@@ -384,10 +421,7 @@ dl_status dl_decode_step_masked(dl_handle *h, const unsigned char *active, const
         if (s != DL_OK) return s;
     }
     const dl_step_io io = {q, k, v, beta, g, out};
-    Lens ln = h->lens;
-    dl_status s = decode_step(h, ln, active, io, static_cast<cudaStream_t>(stream), false, nullptr);
-    if (s == DL_OK) h->lens = std::move(ln);
-    return s;
+    return decode_step(h, h->lens, active, io, static_cast<cudaStream_t>(stream), false, nullptr);
 }
 
 dl_status dl_decode_step(dl_handle *h, const void *q, const void *k, const void *v,
@@ -411,9 +445,11 @@ dl_status dl_merge(dl_handle *h, void *stream) {
             ids.push_back(b);
             lens.push_back(h->lens.of(b));
         }
-    cudaError_t e = launch_slots(h, true, ids, lens, 0, nullptr, h->base, st, false, nullptr);
+    size_t done = 0;
+    cudaError_t e = launch_slots(h, true, ids, lens, 0, nullptr, h->base, st, false, nullptr, &done);
+    for (size_t i = 0; i < done; ++i) h->lens.per[(size_t)ids[i]] = 0;   // merged slots
+    h->lens.join();
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
-    h->lens = Lens();
     return ok();
 }
 
@@ -526,10 +562,16 @@ dl_status dl_cycle_create(dl_handle *const *layers, int n_layers, const dl_step_
         delete cy;
         return fail(DL_ENOMEM, "host allocation of the cycle failed");
     }
-    // with two or more layers on disjoint bases, consecutive kernels of the
-    // token-major cycle belong to different layers: each may start streaming
-    // its base during the previous kernel's tail
-    const bool overlap = n_layers >= 2 && disjoint_bases(layers, n_layers);
+    // with two or more layers that have heads, on disjoint bases,
+    // consecutive kernels of the token-major cycle belong to different
+    // layers (a layer's own consecutive kernels -- slot-list chunks, an
+    // append and its merge -- touch disjoint heads, or the second one is an
+    // ordinary launch): each may start streaming its base during the
+    // previous kernel's tail.  A layer without heads launches nothing, so it
+    // does not separate two steps of another layer.
+    int with_heads = 0;
+    for (int l = 0; l < n_layers; ++l) with_heads += layers[l]->NH > 0 ? 1 : 0;
+    const bool overlap = with_heads >= 2 && disjoint_bases(layers, n_layers);
     cudaStream_t st = nullptr;
     cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
     if (e != cudaSuccess) {
@@ -600,5 +642,7 @@ const char *dl_strerror(dl_status s) {
 }
 
 const char *dl_last_error(void) { return g_err; }
+
+void dl_debug_fake_launches(long long n_ok) { g_fake_ok.store(n_ok < 0 ? -1 : n_ok); }
 
 }  // extern "C"

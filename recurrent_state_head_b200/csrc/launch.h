@@ -74,6 +74,27 @@ cudaError_t allow_smem(std::atomic<unsigned long long> &done, Kernel kern, size_
     return e;
 }
 
+// CTAs of `kern` resident per SM on the current device at `threads`
+// threads and `smem` bytes of dynamic shared memory, computed once per
+// device (callers pass the largest size they launch with, so that the
+// answer does not depend on which launch came first).
+template <typename Kernel>
+cudaError_t resident_ctas(std::atomic<int> (&cache)[64], Kernel kern, int threads, size_t smem, int *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+        if (e != cudaSuccess) return e;
+        n = n > 0 ? n : 1;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return cudaSuccess;
+}
+
 }  // namespace dl
 
 #define DL_DIM_INDEX(d) ((d) == 64 ? 0 : ((d) == 128 ? 1 : -1))
