@@ -320,31 +320,47 @@ def test_no_heads_on_gpu():
 
 # ------------------------------------------------ full-size workloads ----
 
-def _full_size_check(w, n_sample=24, layers=1, T=None, seed=123, mode=B.DL_MERGE_FOLD):
+def _every_head(w, T=None, chunk=1024):
+    """Both merge modes over T tokens of a full-size workload, then every
+    head's outputs (every token) and final materialised state against the
+    oracle's eager recurrence; the oracle runs once, over head chunks, and
+    the per-token error is the normwise-max over all heads."""
     T = w.T if T is None else T
-    rng = np.random.default_rng(seed)
-    heads = np.unique(np.concatenate([[0, w.heads - 1],
-                                      rng.choice(w.heads, n_sample - 2, replace=False)]))
-    for l in range(layers):
-        S0 = synth.initial_state(w, layer=l)
-        bonus = synth.bonus(w, layer=l)
-        ti = synth.tokens(w, 0, T, layer=l, want64=False)
-        x = D.to_device(ti, w)
+    S0 = synth.initial_state(w)
+    bonus = synth.bonus(w)
+    ti = synth.tokens(w, 0, T, want64=False)
+    x = D.to_device(ti, w)
+    runs = []
+    for mode in MODES:
         layer = D.DecodeLayer(w, S0, bonus, auto_merge=mode)
         outs = layer.new_out(T)
         for t in range(T):
             layer.step(x, t, outs[t])
-        mat = layer.materialize()
-        torch.cuda.synchronize()
+        runs.append((outs, layer.materialize(), layer.L))
+        del layer
+    torch.cuda.synchronize()
+    del x
+    for outs, _, L in runs:
         assert torch.isfinite(outs.float()).all()
+        assert L == T % w.C
+    num_o = np.zeros((len(runs), T))
+    den_o = np.zeros(T)
+    num_s = np.zeros(len(runs))
+    den_s = 0.0
+    for h0 in range(0, w.heads, chunk):
+        heads = np.arange(h0, min(w.heads, h0 + chunk))
         Sr, q, k, v, beta, g, bon = oracle_inputs(w, ti, heads=heads, S0=S0, bonus=bonus)
         S_ref, o_ref = run_oracle_eager(w, Sr, q, k, v, beta, g, bon)
-        o = to_np(outs[:, heads])
-        worst = max(rel_err(o[t], o_ref[t]) for t in range(T))
-        assert worst <= tol_out(w), worst
-        assert rel_err(to_np(mat[heads]), S_ref) <= TOL_STATE
-        del x, layer, outs, mat
-        torch.cuda.empty_cache()
+        den_o = np.maximum(den_o, np.abs(o_ref).reshape(T, -1).max(axis=1))
+        den_s = max(den_s, float(np.abs(S_ref).max()))
+        for i, (outs, mat, _) in enumerate(runs):
+            o = to_np(outs[:, h0:h0 + len(heads)])
+            num_o[i] = np.maximum(num_o[i], np.abs(o - o_ref).reshape(T, -1).max(axis=1))
+            num_s[i] = max(num_s[i], float(np.abs(to_np(mat[h0:h0 + len(heads)]) - S_ref).max()))
+    for i, mode in enumerate(MODES):
+        worst = float((num_o[i] / den_o).max())
+        assert worst <= tol_out(w), (mode, worst)
+        assert num_s[i] / den_s <= TOL_STATE, (mode, num_s[i] / den_s)
 
 
 def test_full_gdn_fp32_small():
@@ -367,17 +383,9 @@ def test_full_gdn_fp32_small():
 @pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c4",
                                   "kda-b128-h32-d128-c8", "rwkv6-b128-h32-d64-c4",
                                   "rwkv6-b128-h32-d64-c8"])
-@pytest.mark.parametrize("mode", MODES)
-def test_full_size_256_tokens(name, mode):
-    _full_size_check(synth.WORKLOADS[name], mode=mode)
-
-
-@pytest.mark.parametrize("C", [1, 2, 16])
-def test_stack_largest_batch(C):
-    """The 24-layer GDN stack at its largest batch (B=512: 8192 heads per
-    layer), two of its layers, two cycles and a ragged third."""
-    w = synth.WORKLOADS[f"gdn-stack24-b512-h16-d128-c{C}"]
-    _full_size_check(w, layers=2, T=2 * C + 3)
+def test_full_size_every_head(name):
+    """The full-size workloads, 256 tokens, both merge modes: every head."""
+    _every_head(synth.WORKLOADS[name])
 
 
 @pytest.mark.parametrize("op", OPS)
