@@ -286,15 +286,49 @@ def cpu_oracle_sample(w, target_s=12.0, seed=99, extras=True):
 
 # ------------------------------------------------------------ native ----
 
-def _layers(w, R, rank, dev, mode, xs=None):
-    from recurrent_state_head_b200 import device as D
-    from recurrent_state_head_b200 import synth
-    out = []
-    for l in range(R):
-        lid = rank * R + l
-        out.append(D.DecodeLayer(w, synth.initial_state(w, layer=lid), synth.bonus(w, layer=lid),
-                                 device=dev, auto_merge=mode))
-    return out
+NOMINAL_HBM_GBS = 8000.0          # HBM3e nominal, for context beside the measured copy peak
+SWEEP_B = (1, 8, 32, 128, 512)
+SWEEP_C = (1, 2, 4, 8, 16)
+SWEEP_STEPS = 512
+EXTRA_WORKLOADS = ("kda-b128-h32-d128-c4", "kda-b128-h32-d128-c8",
+                   "rwkv6-b128-h32-d64-c4", "rwkv6-b128-h32-d64-c8")
+
+
+def working_set(w, R):
+    bm = bytes_model(w)
+    return R * w.heads * (bm["S"] + w.C * bm["E"])
+
+
+def workload_config(w, R, world):
+    """The `config` object of a bench line (the same keys in both arms)."""
+    ws = working_set(w, R)
+    l2 = (f"inputs larger than L2: {R} rotating layers, working set {ws / 1e6:.0f} MB vs L2 "
+          f"{L2_BYTES / 1e6:.0f} MB" if ws >= L2_BYTES else
+          f"working set {ws / 1e6:.1f} MB fits in L2 ({L2_BYTES / 1e6:.0f} MB): hot-cache figures")
+    return {"workload": w.name, "op": ["gdn", "kda", "rwkv6"][w.op], "B": w.B, "H": w.H,
+            "dk": w.dk, "dv": w.dv, "C": w.C, "layers_rotated": R,
+            "inputs": f"q/k/v {w.in_dtype}, out {w.out_dtype}, fp32 state", "l2": l2,
+            "step": f"one CUDA-graph merge cycle of {R} layers: {w.C - 1} appends + "
+                    f"1 merge-token per layer, token-major",
+            "parallelism": f"replicas{world}"}
+
+
+class Setup:
+    """States and C tokens of inputs of R independent layers (replica seeds)."""
+
+    def __init__(self, w, R, rank, dev):
+        from recurrent_state_head_b200 import device as D
+        from recurrent_state_head_b200 import synth
+        self.w, self.R, self.dev = w, R, dev
+        ids = [rank * R + l for l in range(R)]
+        self.S0 = [synth.initial_state(w, layer=i) for i in ids]
+        self.bon = [synth.bonus(w, layer=i) for i in ids]
+        self.xs = [D.to_device(synth.tokens(w, 0, w.C, layer=i, want64=False), w, dev) for i in ids]
+
+    def layers(self, mode):
+        from recurrent_state_head_b200 import device as D
+        return [D.DecodeLayer(self.w, self.S0[l], self.bon[l], device=self.dev, auto_merge=mode)
+                for l in range(self.R)]
 
 
 def _ios(w, xs, outs, R, C):
@@ -324,10 +358,12 @@ def kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps, prime, merge_
     The kernels are launched through the C ABI with pointers prepared in
     advance, right after `prime()` (one cycle-graph launch) has queued a
     millisecond of GPU work, so that the host stays ahead of the GPU and the
-    events bracket kernel time only.  layers: decode layers in merge-token
-    mode (each dl_decode_step is one kernel); merge_layers (optional): layers
-    with auto_merge off, for the separate merge kernel (dl_merge)."""
-    import ctypes
+    events bracket kernel time only.  These are isolated launches: inside
+    the cycle graph consecutive kernels overlap their ramp and tail, so the
+    sum of these durations exceeds the graph's step time.  layers: decode
+    layers in merge-token mode (each dl_decode_step is one kernel);
+    merge_layers (optional): layers with auto_merge off, for the separate
+    merge kernel (dl_merge)."""
     import torch
     from recurrent_state_head_b200 import binding as B
     lib = B.lib()
@@ -372,35 +408,42 @@ def kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps, prime, merge_
     return out
 
 
-def run_native(args, rank, world, local_rank):
+def eager_graph(w, states, xs, outs, bons, R, C, stream, dev):
+    """C tokens through R layers of the eager kernel, captured as one graph."""
     import torch
     from recurrent_state_head_b200 import binding as B
     from recurrent_state_head_b200 import device as D
-    from recurrent_state_head_b200 import synth
+    cfg = D.config_of(w)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for t in range(C):
+                for l in range(R):
+                    beta = None if w.op == 2 else xs[l]["beta"][t]
+                    B.dl_eager_step(cfg, states[l], xs[l]["q"][t], xs[l]["k"][t], xs[l]["v"][t],
+                                    beta, xs[l]["g"][t], bons[l], outs[l][t], side)
+    stream.wait_stream(side)
+    return g
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU")
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    init_dist(world, "nccl")
-    B.lib()                                   # fail loudly if the library is missing
 
-    w = synth.WORKLOADS[args.workload]
-    R = args.layers
+def measure(w, R, args, dev, stream, peaks, headline):
+    """Every figure of one workload: the graph-captured merge cycle (timed
+    region), per-kernel durations, the separate-merge and staggered-slot
+    cycles, the eager kernel.  Returns (result dict, objects kept for e2e)."""
+    import torch
+    from recurrent_state_head_b200 import binding as B
+
+    rank = int(os.environ.get("RANK", "0"))
     C, NH = w.C, w.heads
     bm = bytes_model(w, fold=True)
     bm_sep = bytes_model(w, fold=False)
-    stream = torch.cuda.current_stream(dev)
-    peaks = measured_peaks()
-
-    # --- state and inputs of R independent layers (replica-specific seeds)
-    xs = [D.to_device(synth.tokens(w, 0, C, layer=rank * R + l, want64=False), w, dev)
-          for l in range(R)]
-    layers = _layers(w, R, rank, dev, B.DL_MERGE_FOLD)
+    su = Setup(w, R, rank, dev)
+    xs = su.xs
+    layers = su.layers(B.DL_MERGE_FOLD)
     outs = [L_.new_out(C) for L_ in layers]
-    working_set = R * (NH * bm["S"] + NH * C * bm["E"])
     cycle = B.Cycle([L_.handle for L_ in layers], _ios(w, xs, outs, R, C))
-    kernels_per_step = cycle.kernels
 
     # --- timed region: K cycle launches
     for _ in range(args.warmup):
@@ -417,18 +460,17 @@ def run_native(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     barrier(dev)
     torch.cuda.synchronize(dev)
-    elapsed_ms = ev0.elapsed_time(ev1)
     tokens_local = w.B * C * R * args.steps          # decode tokens through one layer
-    max_ms, tokens_all = reduce_over_ranks(elapsed_ms, tokens_local, dev)
+    max_ms, tokens_all = reduce_over_ranks(ev0.elapsed_time(ev1), tokens_local, dev)
     ms_per_step = max_ms / args.steps
-    tok_s = tokens_all / (max_ms / 1e3)
     us_per_token = ms_per_step * 1e3 / (C * R)
     gbs = NH * (bm["token_read"] + bm["token_write"]) * C * R / (ms_per_step / 1e3) / 1e9
 
-    # --- per-kernel durations, CUDA events inside a replayed graph
-    merge_layers = _layers(w, R, rank, dev, B.DL_MERGE_OFF)
+    # --- per-kernel durations (isolated launches)
+    merge_layers = su.layers(B.DL_MERGE_OFF)
     kd = kernel_durations(layers, xs, outs, w, R, C, stream, dev, reps=max(3, min(args.steps, 10)),
                           prime=lambda: cycle.launch(stream), merge_layers=merge_layers)
+    del merge_layers
     app = {t: statistics.mean(kd[("append", t)]) for t in range(C - 1) if ("append", t) in kd}
     fold_us = statistics.mean(kd[("merge_token", C - 1)]) * 1e3 if ("merge_token", C - 1) in kd else None
     merge_us = statistics.mean(kd[("merge", C)]) * 1e3
@@ -441,49 +483,38 @@ def run_native(args, rank, world, local_rank):
         app_bytes = NH * sum(bm["merge_token"](0))
         dominant = "append_kernel (merge-token)"
     achieved = app_bytes / (app_avg_ms / 1e3) / 1e9
-    traffic = recorded_traffic(args.workload)
-
-    result = {
-        "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "op": ["gdn", "kda", "rwkv6"][w.op], "B": w.B,
-                   "H": w.H, "dk": w.dk, "dv": w.dv, "C": C, "layers_rotated": R,
-                   "inputs": f"q/k/v {w.in_dtype}, out {w.out_dtype}, fp32 state",
-                   "l2": f"inputs larger than L2: {R} rotating layers, working set "
-                         f"{working_set / 1e6:.0f} MB vs L2 {L2_BYTES / 1e6:.0f} MB",
-                   "step": f"one CUDA-graph merge cycle of {R} layers: {C - 1} appends + "
-                           f"1 merge-token per layer, token-major",
-                   "parallelism": f"replicas{world}"},
-        "us_per_token": us_per_token,
-        "hbm_gbs": gbs,
-        "hbm_frac": gbs / peaks["hbm_gbs"],
+    res = {
+        "value": tokens_all / (max_ms / 1e3), "ms_per_step": ms_per_step,
+        "us_per_token": us_per_token, "hbm_gbs": gbs,
+        "hbm_frac": gbs / peaks["hbm_gbs"], "hbm_frac_nominal": gbs / NOMINAL_HBM_GBS,
         "bytes_written_per_token": NH * bm["token_write"],
         "bytes_read_per_token": NH * bm["token_read"],
         "kernels": {"append_us_by_L": [app[L] * 1e3 for L in sorted(app)],
                     "append_avg_us": app_avg_ms * 1e3,
                     "merge_token_us": fold_us, "merge_us": merge_us,
-                    "merge_gbs": NH * sum(bm["merge"](C)) / (merge_us / 1e6) / 1e9},
+                    "merge_gbs": NH * sum(bm["merge"](C)) / (merge_us / 1e6) / 1e9,
+                    "timing": "isolated launches, CUDA events between kernels"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": traffic, "kernel": dominant,
-                     "peak_source": peaks["source"]},
-        "gpu_launches": kernels_per_step * args.steps,
+                     "traffic": recorded_traffic(w.name), "kernel": dominant,
+                     "peak_source": peaks["source"], "peak_nominal": NOMINAL_HBM_GBS,
+                     "frac_nominal": achieved / NOMINAL_HBM_GBS,
+                     "timing": "isolated launches of the kernel, mean over the cycle's log "
+                               "lengths, CUDA events on the launching stream"},
+        "gpu_launches": cycle.kernels * args.steps,
         "clocks": clk.summary(),
     }
     if fold_us:
-        result["kernels"]["merge_token_gbs"] = \
-            NH * sum(bm["merge_token"](C - 1)) / (fold_us / 1e6) / 1e9
-    del merge_layers
+        res["kernels"]["merge_token_gbs"] = NH * sum(bm["merge_token"](C - 1)) / (fold_us / 1e6) / 1e9
+        res["kernels"]["merge_token_frac"] = res["kernels"]["merge_token_gbs"] / peaks["hbm_gbs"]
 
     # --- the same cycle with the merge as its own kernel (ablation)
     if args.ablation:
-        sep = _layers(w, R, rank, dev, B.DL_MERGE_SEPARATE)
+        sep = su.layers(B.DL_MERGE_SEPARATE)
         cyc_sep = B.Cycle([L_.handle for L_ in sep], _ios(w, xs, outs, R, C))
         ms = _time_graph(lambda: cyc_sep.launch(stream), stream, args.steps, args.warmup, dev)
-        ms = ms / args.steps
-        result["separate_merge"] = {
+        ms, _ = reduce_over_ranks(ms / args.steps, 0, dev)
+        res["separate_merge"] = {
             "us_per_token": ms * 1e3 / (C * R),
             "hbm_gbs": NH * (bm_sep["token_read"] + bm_sep["token_write"]) * C * R / (ms / 1e3) / 1e9,
             "bytes_written_per_token": NH * bm_sep["token_write"]}
@@ -494,15 +525,15 @@ def run_native(args, rank, world, local_rank):
     #     joined b mod C tokens late), so every token of the cycle runs an
     #     append over 7/8 of the slots and a merge-token over the rest
     if args.staggered and C > 1:
-        stag = _layers(w, R, rank, dev, B.DL_MERGE_FOLD)
+        stag = su.layers(B.DL_MERGE_FOLD)
         for l, L_ in enumerate(stag):
             for t in range(C - 1):
                 L_.step(xs[l], t, outs[l][t], stream=stream,
                         active=[(b % C) > t for b in range(w.B)])
         cyc_st = B.Cycle([L_.handle for L_ in stag], _ios(w, xs, outs, R, C))
         ms = _time_graph(lambda: cyc_st.launch(stream), stream, args.steps, args.warmup, dev)
-        ms = ms / args.steps
-        result["staggered"] = {
+        ms, _ = reduce_over_ranks(ms / args.steps, 0, dev)
+        res["staggered"] = {
             "us_per_token": ms * 1e3 / (C * R),
             "hbm_gbs": gbs * us_per_token / (ms * 1e3 / (C * R)),
             "kernels_per_step": cyc_st.kernels,
@@ -512,61 +543,248 @@ def run_native(args, rank, world, local_rank):
 
     # --- eager dense baseline, same layers and rotation, graph-captured
     if args.eager:
-        cfg = D.config_of(w)
         eager_S = [L_.base.clone() for L_ in layers]
-        bon = [L_.bonus for L_ in layers]
-        g_eager = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g_eager, stream=side):
-                for t in range(C):
-                    for l in range(R):
-                        beta = None if w.op == synth.RWKV6 else xs[l]["beta"][t]
-                        B.dl_eager_step(cfg, eager_S[l], xs[l]["q"][t], xs[l]["k"][t],
-                                        xs[l]["v"][t], beta, xs[l]["g"][t], bon[l],
-                                        outs[l][t], side)
-        stream.wait_stream(side)
+        g_eager = eager_graph(w, eager_S, xs, outs, [L_.bonus for L_ in layers], R, C, stream, dev)
         e_ms = _time_graph(g_eager.replay, stream, args.steps, args.warmup, dev) / args.steps
+        e_ms, _ = reduce_over_ranks(e_ms, 0, dev)
         e_read, e_write = bm["eager"]
-        result["eager"] = {
+        res["eager"] = {
             "us_per_token": e_ms * 1e3 / (C * R),
-            "tok_s": w.B * C * R / (e_ms / 1e3),
+            "tok_s": w.B * C * R * world_size() / (e_ms / 1e3),
             "hbm_gbs": NH * (e_read + e_write) * C * R / (e_ms / 1e3) / 1e9,
             "bytes_written_per_token": NH * e_write,
             "write_ratio_vs_deltalog": e_write / bm["token_write"],
             "speedup_deltalog": (e_ms * 1e3 / (C * R)) / us_per_token,
         }
-        result["eager"]["hbm_frac"] = result["eager"]["hbm_gbs"] / peaks["hbm_gbs"]
+        res["eager"]["hbm_frac"] = res["eager"]["hbm_gbs"] / peaks["hbm_gbs"]
         del g_eager, eager_S
+    keep = {"setup": su, "layers": layers, "outs": outs, "cycle": cycle, "tokens_local": tokens_local}
+    return res, keep
 
-    # --- end to end through the public API with host buffers
-    if args.e2e:
-        names = ("q", "k", "v", "beta", "g")
-        host_in = [{n: xs[l][n].cpu().pin_memory() for n in names} for l in range(R)]
-        host_out = [torch.empty(outs[l].shape, dtype=outs[l].dtype).pin_memory()
-                    for l in range(R)]
-        h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
-        d2h = sum(t.numel() * t.element_size() for t in host_out)
 
-        def e2e_step():
+def world_size():
+    return int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def e2e_overlapped(w, R, keep, args, dev, stream):
+    """End to end through the public API with host buffers: every step
+    copies that step's inputs from pinned host memory, launches the cycle
+    (dl_cycle_launch) and copies the outputs back to pinned host memory.
+    Two device buffer sets alternate, with a cycle graph captured over each,
+    so the inputs of step k+1 (one copy stream) and the outputs of step k-1
+    (another) cross PCIe while step k computes; events order each buffer's
+    reuse.  The timed region runs from before the first copy to after the
+    last one, on the launching stream."""
+    import torch
+    from recurrent_state_head_b200 import binding as B
+    names = ("q", "k", "v", "beta", "g")
+    su, layers = keep["setup"], keep["layers"]
+    C = w.C
+    host_in = [{n: su.xs[l][n].cpu().pin_memory() for n in names} for l in range(R)]
+    sets = []
+    for s in range(2):
+        xs_s = [{n: torch.empty_like(su.xs[l][n]) for n in names} for l in range(R)]
+        outs_s = [L_.new_out(C) for L_ in layers]
+        cyc = B.Cycle([L_.handle for L_ in layers], _ios(w, xs_s, outs_s, R, C))
+        host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs_s]
+        sets.append((xs_s, outs_s, cyc, host_out))
+    h2d_bytes = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
+    d2h_bytes = sum(t.numel() * t.element_size() for t in sets[0][3])
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ev_in, ev_done, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def load(s):
+        with torch.cuda.stream(h2d):
             for l in range(R):
                 for n in names:
-                    xs[l][n].copy_(host_in[l][n], non_blocking=True)
-            cycle.launch(stream)
-            for l in range(R):
-                host_out[l].copy_(outs[l], non_blocking=True)
+                    sets[s][0][l][n].copy_(host_in[l][n], non_blocking=True)
+            ev_in[s].record(h2d)
 
-        barrier(dev)
-        e_ms = _time_graph(e2e_step, stream, args.steps, max(1, args.warmup), dev)
-        barrier(dev)
-        e_max, e_tok = reduce_over_ranks(e_ms, tokens_local, dev)
-        result["e2e"] = {"value": e_tok / (e_max / 1e3), "unit": "tok/s",
-                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    def run(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d.wait_stream(stream)
+        d2h.wait_stream(stream)
+        load(0)
+        for k in range(K):
+            s = k % 2
+            if k + 1 < K:
+                s1 = (k + 1) % 2
+                if k >= 1:
+                    h2d.wait_event(ev_done[s1])       # step k-1 has read set s1
+                load(s1)
+            stream.wait_event(ev_in[s])
+            if k >= 2:
+                stream.wait_event(ev_out[s])          # step k-2's outputs are out
+            sets[s][2].launch(stream)
+            ev_done[s].record(stream)
+            d2h.wait_event(ev_done[s])
+            with torch.cuda.stream(d2h):
+                for l in range(R):
+                    sets[s][3][l].copy_(sets[s][1][l], non_blocking=True)
+                ev_out[s].record(d2h)
+        stream.wait_stream(d2h)
+        stream.wait_stream(h2d)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    run(max(3, args.warmup))
+    barrier(dev)
+    e_ms = run(args.steps)
+    barrier(dev)
+    e_max, e_tok = reduce_over_ranks(e_ms, keep["tokens_local"], dev)
+    for s in sets:
+        s[2].close()
+    return {"value": e_tok / (e_max / 1e3), "unit": "tok/s",
+            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+            "ms_per_step": e_max / args.steps,
+            "note": "pinned host inputs in, outputs out every step; two buffer sets, copies "
+                    "on two copy streams overlapping the previous / next step's cycle"}
+
+
+def run_sweep(args, dev, stream, peaks):
+    """The 24-layer GDN stack (heads of the B128 H16 d128 workload), one
+    decode step per layer in sequence, for every (B, C) cell: 512 steps per
+    layer as 512 / C launches of one cycle graph over the stack.  Stacks
+    smaller than 4x L2 are replicated and the replicas decoded in turn, so
+    that every base read comes from HBM (hot figures, one stack, alongside).
+    States and inputs are drawn on the device (torch's generator, the
+    workloads' distributions): 12 GB of state at B = 512 is too much to
+    draw on the host in a benchmark."""
+    import torch
+    from recurrent_state_head_b200 import binding as B
+    from recurrent_state_head_b200 import device as D
+    from recurrent_state_head_b200 import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4_000 + rank)
+    cells = []
+    steps, warm = SWEEP_STEPS, max(3, args.warmup)
+    with ClockSampler(dev) as clk:
+        for Bsz in SWEEP_B:
+            w16 = synth.WORKLOADS[f"gdn-stack24-b{Bsz}-h16-d128-c16"]
+            NH, nl = w16.heads, w16.layers
+            stack_state = nl * NH * 4 * w16.dk * w16.dv
+            reps = max(1, math.ceil(4 * L2_BYTES / stack_state))
+            R = nl * reps
+            bases = [D.draw_state(w16, l, dev, gen) for l in range(R)]
+            xs = [D.draw_tokens(w16, max(SWEEP_C), dev, gen) for l in range(R)]
+            outs = [torch.empty((max(SWEEP_C), NH, w16.dv), dtype=torch.bfloat16, device=dev)
+                    for _ in range(R)]
+            for C in SWEEP_C:
+                w = synth.WORKLOADS[f"gdn-stack24-b{Bsz}-h16-d128-c{C}"]
+                bm = bytes_model(w)
+                layers = [D.DecodeLayer(w, bases[l], None, device=dev) for l in range(R)]
+                cyc = B.Cycle([L_.handle for L_ in layers], _ios(w, xs, outs, R, C))
+                n = steps // C
+                ms = _time_graph(lambda: cyc.launch(stream), stream, n, warm, dev)
+                ms, _ = reduce_over_ranks(ms, 0, dev)
+                us = ms * 1e3 / (n * C * R)
+                cell = {"B": Bsz, "C": C, "state_MB_per_stack": stack_state / 2 ** 20,
+                        "replicas": reps, "deltalog_us_per_token": us,
+                        "deltalog_gbs": NH * (bm["token_read"] + bm["token_write"]) / us / 1e3,
+                        "deltalog_write_bytes_per_token": NH * bm["token_write"],
+                        "kernels_per_launch": cyc.kernels}
+                cell["deltalog_hbm_frac"] = cell["deltalog_gbs"] / peaks["hbm_gbs"]
+                if reps > 1:
+                    hot = B.Cycle([L_.handle for L_ in layers[:nl]], _ios(w, xs, outs, nl, C))
+                    hms = _time_graph(lambda: hot.launch(stream), stream, n, warm, dev)
+                    hms, _ = reduce_over_ranks(hms, 0, dev)
+                    cell["deltalog_us_per_token_hot"] = hms * 1e3 / (n * C * nl)
+                    hot.close()
+                cyc.close()
+                del layers
+                g = eager_graph(w, bases, xs, outs, [None] * R, R, C, stream, dev)
+                ems = _time_graph(g.replay, stream, n, warm, dev)
+                ems, _ = reduce_over_ranks(ems, 0, dev)
+                e_read, e_write = bm["eager"]
+                eus = ems * 1e3 / (n * C * R)
+                cell.update({"eager_us_per_token": eus,
+                             "eager_gbs": NH * (e_read + e_write) / eus / 1e3,
+                             "eager_write_bytes_per_token": NH * e_write,
+                             "speedup": eus / us, "write_ratio": e_write / bm["token_write"]})
+                del g
+                cells.append(cell)
+            del bases, xs, outs
+            torch.cuda.empty_cache()
+    return {"steps": steps, "layers": 24, "cells": cells, "clocks": clk.summary(),
+            "unit": "µs per layer-token (amortised over the cycle)",
+            "inputs": "device-drawn (torch Philox), workload distributions; C tokens of inputs "
+                      "reused every launch"}
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    from recurrent_state_head_b200 import binding as B
+    from recurrent_state_head_b200 import synth
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    B.lib()                                   # fail loudly if the library is missing
+
+    w = synth.WORKLOADS[args.workload]
+    R = args.layers
+    stream = torch.cuda.current_stream(dev)
+    peaks = measured_peaks()
+    res, keep = measure(w, R, args, dev, stream, peaks, headline=True)
+    result = {
+        "metric": METRIC, "value": res.pop("value"), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic", "config": workload_config(w, R, world),
+    }
+    result.update(res)
+    if args.e2e:
+        result["e2e"] = e2e_overlapped(w, R, keep, args, dev, stream)
+    keep["cycle"].close()
+    del keep
+    torch.cuda.empty_cache()
+
+    # --- the other operators at one GPU (GDN, KDA, RWKV6 at C = 4 and 8)
+    if args.workloads:
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            wx = synth.WORKLOADS[name]
+            r, k = measure(wx, R, args, dev, stream, peaks, headline=False)
+            k["cycle"].close()
+            del k
+            torch.cuda.empty_cache()
+            extra[name] = {
+                "us_per_token": r["us_per_token"], "tok_s": r["value"], "hbm_gbs": r["hbm_gbs"],
+                "hbm_frac": r["hbm_frac"], "hbm_frac_nominal": r["hbm_frac_nominal"],
+                "append_avg_us": r["kernels"]["append_avg_us"],
+                "append_roofline_frac": r["roofline"]["frac"],
+                "merge_token_us": r["kernels"]["merge_token_us"],
+                "merge_token_frac": r["kernels"].get("merge_token_frac"),
+                "merge_us": r["kernels"]["merge_us"],
+                "bytes_written_per_token": r["bytes_written_per_token"],
+                "clocks": r["clocks"],
+            }
+            if "eager" in r:
+                extra[name].update({"eager_us_per_token": r["eager"]["us_per_token"],
+                                    "eager_hbm_frac": r["eager"]["hbm_frac"],
+                                    "write_ratio": r["eager"]["write_ratio_vs_deltalog"],
+                                    "speedup": r["eager"]["speedup_deltalog"]})
+            if "separate_merge" in r:
+                extra[name]["separate_merge_us_per_token"] = r["separate_merge"]["us_per_token"]
+            if "staggered" in r:
+                extra[name]["staggered_us_per_token"] = r["staggered"]["us_per_token"]
+        result["workloads"] = extra
+
+    # --- the 24-layer stack: state-size and interval sweep
+    if args.sweep:
+        result["sweep"] = run_sweep(args, dev, stream, peaks)
 
     if rank == 0 and world == 1 and args.cpu_baseline:
         result["cpu_baseline"] = cpu_oracle_sample(w)
-    cycle.close()
     return result
 
 
@@ -596,9 +814,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "op": ["gdn", "kda", "rwkv6"][w.op], "B": w.B,
-                   "H": w.H, "dk": w.dk, "dv": w.dv, "C": w.C,
-                   "parallelism": "host cores (oracle)"},
+        "config": workload_config(w, args.layers, world),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": last["cores"],
                          "kind": "oracle", "sample": last["sample"]},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
@@ -621,6 +837,10 @@ def main(argv=None):
     ap.add_argument("--no-ablation", dest="ablation", action="store_false",
                     help="skip the separate-merge cycle")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-workloads", dest="workloads", action="store_false",
+                    help="skip the KDA and RWKV6 workloads")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false",
+                    help="skip the 24-layer stack sweep")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args(argv)
     if args.warmup < 3:

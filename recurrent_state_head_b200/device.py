@@ -50,14 +50,22 @@ def config_of(w: Workload, C=None, auto_merge=1) -> B.dl_config:
 
 
 class DecodeLayer:
-    """One layer of DeltaLog decode state on the GPU."""
+    """One layer of DeltaLog decode state on the GPU.  S0 is the starting
+    dense state: a host array (copied to the device), or a float32 device
+    tensor of NH * dk * dv elements, used as the base itself (not copied)."""
 
-    def __init__(self, w: Workload, S0: np.ndarray, bonus=None, device="cuda", C=None,
+    def __init__(self, w: Workload, S0, bonus=None, device="cuda", C=None,
                  auto_merge=1):
         self.w = w
         self.cfg = config_of(w, C, auto_merge)
-        self.base = torch.from_numpy(np.ascontiguousarray(S0, dtype=np.float32)).reshape(
-            w.heads, w.dk, w.dv).to(device)
+        if isinstance(S0, torch.Tensor):
+            if S0.dtype != torch.float32 or S0.numel() != w.heads * w.dk * w.dv:
+                raise ValueError("device base must be float32 with NH * dk * dv elements")
+            self.base = S0.reshape(w.heads, w.dk, w.dv)
+            device = S0.device
+        else:
+            self.base = torch.from_numpy(np.ascontiguousarray(S0, dtype=np.float32)).reshape(
+                w.heads, w.dk, w.dv).to(device)
         self.log = torch.zeros(max(B.dl_log_bytes(self.cfg), 16), dtype=torch.uint8,
                                device=device)
         self.bonus = (torch.from_numpy(np.ascontiguousarray(bonus, dtype=np.float32)).to(device)
@@ -117,3 +125,41 @@ def eager_step(w: Workload, S: torch.Tensor, x: dict, t: int, bonus, out, stream
     beta = None if w.op == RWKV6 else x["beta"][t]
     B.dl_eager_step(cfg, S, x["q"][t], x["k"][t], x["v"][t], beta, x["g"][t], bonus, out,
                     stream)
+
+
+# ---------------------------------------------- device-drawn timing inputs --
+
+def draw_state(w: Workload, layer: int, device, generator: torch.Generator) -> torch.Tensor:
+    """A starting state [NH, dk, dv] drawn on the device with the workload's
+    distribution (N(0, init_std), or zero), for timing runs too large to draw
+    on the host.  Torch's device generator, not synth's: these values never
+    meet the checker."""
+    shape = (w.heads, w.dk, w.dv)
+    if w.init_std == 0.0:
+        return torch.zeros(shape, dtype=torch.float32, device=device)
+    S = torch.empty(shape, dtype=torch.float32, device=device)
+    S.normal_(0.0, w.init_std, generator=generator)
+    return S
+
+
+def draw_tokens(w: Workload, n: int, device, generator: torch.Generator) -> dict:
+    """n tokens of inputs drawn on the device with synth's distributions
+    (q, k, v ~ N(0, 1), q and k L2-normalised for GDN/KDA; beta =
+    sigmoid(N(0, 1)); g = -softplus(N(0, 1)) for GDN/KDA, -exp(N(-0.5, 0.5))
+    for RWKV6), rounded to the workload's dtypes; laid out as to_device's."""
+    NH = w.heads
+    f = dict(dtype=torch.float32, device=device)
+    q = torch.randn((n, NH, w.dk), generator=generator, **f)
+    k = torch.randn((n, NH, w.dk), generator=generator, **f)
+    v = torch.randn((n, NH, w.dv), generator=generator, **f)
+    x = torch.randn((n, NH, w.m), generator=generator, **f)
+    if w.op == RWKV6:
+        beta = torch.zeros((n, NH), **f)
+        g = -torch.exp(x * 0.5 - 0.5)
+    else:
+        beta = torch.sigmoid(torch.randn((n, NH), generator=generator, **f))
+        g = -torch.nn.functional.softplus(x)
+        q = q / q.norm(dim=-1, keepdim=True)
+        k = k / k.norm(dim=-1, keepdim=True)
+    t = TORCH_DTYPE[w.in_dtype]
+    return {"q": q.to(t), "k": k.to(t), "v": v.to(t), "beta": beta, "g": g}
