@@ -89,18 +89,34 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
     return launch_tv<OP, DK, DV, 32, FOLD>(p, s);
 }
 
-// Slot list: p.L is the longest length in the list.
-template <int OP, int DK, int DV, int TV>
-cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
-    constexpr int NT = CtaShape<DK, TV>::NT;
+// Slot list: p.L is the longest length in the list; the merge-token
+// entries (the first sl.nfold) are all at that length, one short of full.
+// Merge-token units use 32-column tiles, so that the thread count of the
+// append's shape gives them 8 rows a thread.
+template <int OP, int DK, int DV, int TVA, int LB>
+cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+    constexpr int TVF = 32;
+    constexpr int NT = AppendShape<DK, TVA, false>::NT;
+    static_assert(TVF <= NT && DK <= NT && (DK / (NT / (TVF / 4))) == 8, "merge-token tile shape");
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = append_slots_kernel<OP, DK, DV, TV, NT>;
+    auto kern = append_slots_kernel<OP, DK, DV, TVA, TVF, NT, LB>;
     const int ie = p.in_bf16 ? 2 : 4;
-    const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, sl.nfold > 0).bytes;
-    cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC - 1, 4, true, true).bytes);
+    const size_t sa = op_layout<OP, DK, TVA>(p.L, ie, true, false).bytes;
+    const size_t sf = op_layout<OP, DK, TVF>(p.L, ie, true, true).bytes;
+    const size_t smem = sl.nfold > 0 && sf > sa ? sf : sa;
+    const size_t ma = op_layout<OP, DK, TVA>(MAXC - 1, 4, true, false).bytes;
+    const size_t mf = op_layout<OP, DK, TVF>(MAXC - 1, 4, true, true).bytes;
+    cudaError_t e = allow_smem(smem_ok, kern, ma > mf ? ma : mf);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((long long)sl.n * p.H * (DV / TV));
-    return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p, sl);
+    const long long units = (long long)sl.nfold * p.H * (DV / TVF) + (long long)(sl.n - sl.nfold) * p.H * (DV / TVA);
+    return launch_kernel(kern, (unsigned)units, NT, smem, p.early != 0, s, p, sl);
+}
+
+template <int OP, int DK, int DV, int TVA>
+cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+    if (sl.nfold > 0 && p.L <= 3) return launch_slots_lb<OP, DK, DV, TVA, 3>(p, sl, s);
+    if (sl.nfold > 0 && p.L <= 7) return launch_slots_lb<OP, DK, DV, TVA, 7>(p, sl, s);
+    return launch_slots_lb<OP, DK, DV, TVA, 0>(p, sl, s);
 }
 
 template <int OP, int DK, int DV>

@@ -176,10 +176,11 @@ __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
 // append kernel: the read-once base stream is marked evict-first, so that it
 // does not push out of L2 what the next decode token reads again -- the log
 // entries, written and read evict-last while the log is live.  The
-// merge-token reads and writes everything evict-first (its log is dropped).
-// Measured on B200 in a four-layer merge cycle: 1.4 % (GDN) to 3.7 %
-// (RWKV6) faster than without hints; the merge kernel, whose every byte is
-// touched once, is faster without them and uses none.
+// merge-token reads its log evict-first (the log is dropped after it) and
+// its base tile, read and written back, without a policy.  Measured on B200
+// in a four-layer merge cycle: 1.4 % (GDN) to 3.7 % (RWKV6) faster than
+// without hints; the kernels that read and write the state tile (merge,
+// merge-token) are faster without hints on it.
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -255,6 +256,13 @@ __device__ __forceinline__ void fma4(float4 &acc, float w, const float4 &s) {
     const float2 lo = __ffma2_rn(ww, make_float2(s.x, s.y), make_float2(acc.x, acc.y));
     const float2 hi = __ffma2_rn(ww, make_float2(s.z, s.w), make_float2(acc.z, acc.w));
     acc = make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// s + w * t on four lanes
+__device__ __forceinline__ float4 fma4_ret(const float4 &s, float w, const float4 &t) {
+    float4 o = s;
+    fma4(o, w, t);
+    return o;
 }
 
 // a * s + b * t on four lanes
@@ -550,20 +558,15 @@ __device__ __forceinline__ float4 fold_row_reg(float4 s, float gm, const float *
 // (d_j with q) and the self term k.q (RWKV6: r.(bonus*k)).  AppendDecode:
 // x = Sbar^T w over the register tile (the one base read), value-side replay,
 // delta correction, output.
-// FOLD = false (append, "Fase di Append"): u_t, k_t and Lambda_t go to log
-//   slot L; the base is not written.
-// FOLD = true (merge-token, the step that completes the log: "Fase di
-//   Merge"): the logical state after this token -- base decayed to Lambda_t,
-//   all L logged factors and this token's k u^T -- is written over the base
-//   tile (the register tile is read once and written once); the log is left
-//   for the caller to reset (L = 0).
+// ("Fase di Append"): u_t, k_t and Lambda_t go to log slot L; the base is
+// not written.
 //
 // append_unit does one unit (head, value tile vt) at log length L;
-// append_kernel runs it over all heads at the shared length p.L, and
-// append_slots_kernel over a slot list whose first nfold entries take the
-// merge-token and the rest the append (one launch per step however the
-// slots' lengths are spread).
-template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB>
+// append_kernel runs it (or merge_token_unit, below) over all heads at the
+// shared length p.L, and append_slots_kernel over a slot list whose first
+// nfold entries take the merge-token and the rest the append (one launch per
+// step however the slots' lengths are spread).
+template <int OP, int DK, int DV, int TV, int NT>
 __device__ __forceinline__ void append_unit(const AppendParams &p, const int head, const int vt,
                                             const int L) {
     using T = Tile<DK, DV, TV, NT>;
@@ -578,18 +581,16 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
     __shared__ float s_q[DK];
     __shared__ float s_w[NA][DK];        // read-out weights
     __shared__ float s_bk[OP == OP_RWKV6 ? DK : 1];
-    __shared__ float s_gam[FOLD ? DK : 1];
     __shared__ float s_coef[NA][MAXC];   // replay coefficients (c_j, d_j)
     __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
     __shared__ __align__(16) float s_red[NA * T::NW * TV];
-    __shared__ __align__(16) float s_u[FOLD ? TV : 4];
 
     const int tid = threadIdx.x;
     const int C = p.C;
     const int ie = p.in_bf16 ? 2 : 4;
     const int col4 = tid % T::TPR, rg = tid / T::TPR;
     const int c4 = col4 * 4;
-    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, FOLD);
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, false);
 
     // 1. the base stream: RPT rows x 16 bytes per thread.  As a programmatic
     //    dependent launch (merge cycles over several layers) the stream
@@ -601,9 +602,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
     float4 s[T::RPT];
     auto load_base = [&]() {
 #pragma unroll
-        for (int r = 0; r < T::RPT; ++r)
-            s[r] = FOLD ? ld_state_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first)
-                        : ld_stream_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first);
+        for (int r = 0; r < T::RPT; ++r) s[r] = ld_stream_hint(bh + (size_t)(rg + r * T::RG) * DV, pol_first);
     };
     if (p.early) load_base();
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -613,8 +612,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
     // 2. small operands, staged by warp 0 while the base loads are in flight
     if (tid < 32) {
         const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
-        stage_ops<OP, DK, DV, TV, true>(dsm, lay, src, head, vt, L, C, p.H, ie, true,
-                                        FOLD ? pol_first : pol_last);
+        stage_ops<OP, DK, DV, TV, true>(dsm, lay, src, head, vt, L, C, p.H, ie, true, pol_last);
     }
     __syncthreads();
     const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
@@ -641,7 +639,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             s_w[0][i] = gam * kf;
             s_w[NA - 1][i] = gam * qf;
         }
-        if (!FOLD && vt == 0) {
+        if (vt == 0) {
             copy_raw_hint(p.logK, ((size_t)head * C + L) * DK + i, dsm + lay.kin, i, p.in_bf16, pol_last);
             if (OP != OP_GDN || i == 0) st_f32_hint(p.logLam + ((size_t)head * C + L) * M + x, lt, pol_last);
         }
@@ -681,8 +679,6 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             }
         }
     }
-    if (FOLD) replay_table<OP, DK, NT>(reinterpret_cast<float *>(dsm + lay.A), s_gam, s_lt,
-                                       dsm + lay.K, slam, L, p.in_bf16);
     __syncthreads();
 
     // 4. base read-out: x_a[c] = sum_i w_a[i] * Sbar[i][c]
@@ -715,10 +711,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
                 rr = fmaf(s_coef[0][j], ld_raw(dsm + lay.U, j * TV + c, p.in_bf16), rr);
             const float o = p.scale * (xc[0] + rr + s_self * vv);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-            if (FOLD)
-                s_u[c] = vv;
-            else
-                copy_raw_hint(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16, pol_last);
+            copy_raw_hint(p.logU, ub + (size_t)L * DV, dsm + lay.vin, c, p.in_bf16, pol_last);
         } else {
             const float *U = reinterpret_cast<const float *>(dsm + lay.U);
             float rk = 0.f, rq = 0.f;
@@ -731,42 +724,168 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
             const float u = beta * (vv - xc[0] - rk);
             const float o = p.scale * (xc[NA - 1] + rq + s_self * u);
             st_out(p.out, (size_t)head * DV + col, o, p.out_bf16);
-            if (FOLD)
-                s_u[c] = u;
-            else
-                st_f32_hint(reinterpret_cast<float *>(p.logU) + ub + (size_t)L * DV, u, pol_last);
+            st_f32_hint(reinterpret_cast<float *>(p.logU) + ub + (size_t)L * DV, u, pol_last);
         }
     }
+}
 
-    // 6. merge-token: write the logical state after this token over the base
-    if (FOLD) {
-        __syncthreads();
-        const float *A = reinterpret_cast<const float *>(dsm + lay.A);
-        const int AP = up4(L) + 4;
-        const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-        const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
-        if constexpr (LB > 0) {
-            // the logged value factors of this thread's columns, once
-            float4 ur[LB];
+// ====================================================== merge-token ==
+//
+// The token that completes the log ("Fase di Merge"): the logical state
+// after this token is written over the base tile, which is read once and
+// written once; the log is left for the caller to reset (L = 0).  Since the
+// whole log has to be replayed into the tile anyway, the tile is folded
+// first -- base decayed to the decay point plus every logged factor,
+// S' = D(e^{Lambda_r}) Sbar + sum_j D(e^{Lambda_r - Lambda_j}) k_j u_j^T, with
+// Lambda_r = Lambda_t (GDN/KDA) or Lambda_{t-1} (RWKV6) -- and read out from
+// there, so the replay coefficients and the value-side replay of the append
+// are not needed:
+//   GDN/KDA  x_k = S'^T k, x_q = S'^T q, u = beta (v - x_k),
+//            o = scale (x_q + (k.q) u),  S_t = S' + k u^T
+//   RWKV6    o = scale (S'^T r + (r.(bonus*k)) v),  S_t = D(e^{g_t}) S' + k v^T
+// LB > 0 keeps the L <= LB logged value factors of the thread's columns in
+// registers; LB = 0 reads them from shared memory per row.
+template <int OP, int DK, int DV, int TV, int NT, int LB>
+__device__ __forceinline__ void merge_token_unit(const AppendParams &p, const int head, const int vt,
+                                                 const int L) {
+    using T = Tile<DK, DV, TV, NT>;
+    constexpr int M = (OP == OP_GDN) ? 1 : DK;
+    constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
+    static_assert(TV <= NT && DK <= NT, "one thread per key row and per value column");
+
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ float s_gam[DK];          // decay of the base to the decay point
+    __shared__ float s_w[NA][DK];        // read-out weights: k, q (GDN/KDA) or r (RWKV6)
+    __shared__ float s_k[DK];
+    __shared__ float s_a[OP == OP_RWKV6 ? DK : 1];   // RWKV6: this token's decay e^{g_t}
+    __shared__ float s_self;             // k.q (GDN/KDA) or r.(bonus*k) (RWKV6)
+    __shared__ __align__(16) float s_red[NA * T::NW * TV];
+    __shared__ __align__(16) float s_u[TV];
+
+    const int tid = threadIdx.x;
+    const int ie = p.in_bf16 ? 2 : 4;
+    const int col4 = tid % T::TPR, rg = tid / T::TPR;
+    const int c4 = col4 * 4;
+    const OpLayout lay = op_layout<OP, DK, TV>(L, ie, true, true);
+
+    // 1. the base tile (read and written back: coherent loads, no L2 policy
+    //    -- an evict-first hint on this read-write tile measured 2-4 % slower
+    //    on B200), streamed before the wait on the previous kernel when that
+    //    one cannot be writing this base (see append_unit)
+    float *bh = const_cast<float *>(p.base) + (size_t)head * DK * DV + vt * TV + c4;
+    const uint64_t pol_first = l2_evict_first();
+    float4 s[T::RPT];
+    auto load_base = [&]() {
 #pragma unroll
-            for (int j = 0; j < LB; ++j)
-                ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const int row = rg + r * T::RG;
-                float4 o = fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L);
-                fma4(o, s_k[row], u4);
-                st_state_hint(bh + (size_t)row * DV, o, pol_first);
-            }
+        for (int r = 0; r < T::RPT; ++r) s[r] = ld_state(bh + (size_t)(rg + r * T::RG) * DV);
+    };
+    if (p.early) load_base();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!p.early) load_base();
+
+    // 2. small operands and the log, staged by warp 0 (read once: evict-first)
+    if (tid < 32) {
+        const OpSources src{p.k, p.q, p.v, p.g, p.beta, p.bonus, p.logK, p.logU, p.logLam};
+        stage_ops<OP, DK, DV, TV, true>(dsm, lay, src, head, vt, L, p.C, p.H, ie, true, pol_first);
+    }
+    __syncthreads();
+    const float *sg = reinterpret_cast<const float *>(dsm + lay.g);
+    const float *slam = reinterpret_cast<const float *>(dsm + lay.lam);
+    float *A = reinterpret_cast<float *>(dsm + lay.A);
+    const int AP = up4(L) + 4;
+
+    // 3. replay-factor table A[i][j] = e^{Lambda_r[i] - Lambda_j[i]} k_j[i],
+    //    base decay, read-out weights (all threads); the self term (warp 0)
+    for (int idx = tid; idx < DK * (L + 1); idx += NT) {
+        const int i = idx % DK, j = idx / DK;
+        const int x = (OP == OP_GDN) ? 0 : i;
+        const float lprev = L > 0 ? slam[(L - 1) * M + x] : 0.f;
+        const float lr = (OP == OP_RWKV6) ? lprev : lprev + sg[x];
+        if (j < L) {
+            A[i * AP + j] = expf(lr - slam[j * M + x]) * ld_raw(dsm + lay.K, j * DK + i, p.in_bf16);
         } else {
-#pragma unroll
-            for (int r = 0; r < T::RPT; ++r) {
-                const int row = rg + r * T::RG;
-                float4 o = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-                fma4(o, s_k[row], u4);
-                st_state_hint(bh + (size_t)row * DV, o, pol_first);
-            }
+            const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
+            const float qf = ld_raw(dsm + lay.qin, i, p.in_bf16);
+            s_gam[i] = expf(lr);
+            s_k[i] = kf;
+            s_w[0][i] = (OP == OP_RWKV6) ? qf : kf;
+            s_w[NA - 1][i] = qf;
+            if (OP == OP_RWKV6) s_a[i] = expf(sg[i]);
         }
+    }
+    if (tid < 32) {
+        float a0 = 0.f;
+#pragma unroll
+        for (int i = tid; i < DK; i += 32) {
+            const float kf = ld_raw(dsm + lay.kin, i, p.in_bf16);
+            const float other = (OP == OP_RWKV6) ? reinterpret_cast<const float *>(dsm + lay.bonus)[i] * kf : kf;
+            a0 = fmaf(ld_raw(dsm + lay.qin, i, p.in_bf16), other, a0);
+        }
+        a0 = warp_sum(a0);
+        if (tid == 0) s_self = a0;
+    }
+    __syncthreads();
+
+    // 4. fold the log into the tile, then (a second pass, so that the logged
+    //    factors and the accumulators are not live together) read out
+    //    x_a[c] = sum_i w_a[i] S'[i][c]
+    const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
+    if constexpr (LB > 0) {
+        float4 ur[LB];
+#pragma unroll
+        for (int j = 0; j < LB; ++j)
+            ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            s[r] = fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+            s[r] = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
+        }
+    }
+    float xc[NA];
+    {
+        float4 acc[NA];
+#pragma unroll
+        for (int a = 0; a < NA; ++a) acc[a] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < T::RPT; ++r) {
+            const int row = rg + r * T::RG;
+#pragma unroll
+            for (int a = 0; a < NA; ++a) fma4(acc[a], s_w[a][row], s[r]);
+        }
+        reduce_cols<NA, TV, NT>(acc, s_red, xc);
+    }
+
+    // 5. value side: delta correction (GDN/KDA), output
+    if (tid < TV) {
+        const int c = tid;
+        const int col = vt * TV + c;
+        const float vv = ld_raw(dsm + lay.vin, c, p.in_bf16);
+        if (OP == OP_RWKV6) {
+            st_out(p.out, (size_t)head * DV + col, p.scale * (xc[0] + s_self * vv), p.out_bf16);
+            s_u[c] = vv;
+        } else {
+            const float beta = *reinterpret_cast<const float *>(dsm + lay.beta);
+            const float u = beta * (vv - xc[0]);
+            st_out(p.out, (size_t)head * DV + col, p.scale * (xc[NA - 1] + s_self * u), p.out_bf16);
+            s_u[c] = u;
+        }
+    }
+    __syncthreads();
+
+    // 6. the state after this token over the base tile
+    const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[c4]);
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) {
+        const int row = rg + r * T::RG;
+        const float4 o = (OP == OP_RWKV6) ? fma4_2(s_a[row], s[r], s_k[row], u4) : fma4_ret(s[r], s_k[row], u4);
+        st_state(bh + (size_t)row * DV, o);
     }
 }
 
@@ -780,24 +899,39 @@ append_kernel(const AppendParams p, const Stagger st) {
     if (st.ns > 0 && (int)blockIdx.x < st.slots * st.sms)
         __nanosleep((unsigned)((int)blockIdx.x / st.sms) * (unsigned)st.ns);
     const int lh = (int)blockIdx.x / T::NVT;
-    append_unit<OP, DK, DV, TV, NT, FOLD, LB>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
+    if constexpr (FOLD)
+        merge_token_unit<OP, DK, DV, TV, NT, LB>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
+    else
+        append_unit<OP, DK, DV, TV, NT>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
 }
 
-// The merge-token entries come first, so that their longer CTAs start in
-// the first wave rather than in the tail.  Both paths read the logged value
-// factors from shared memory (LB = 0) and the kernel is held to the
-// append's 64 registers, so that it keeps the append's occupancy.
-template <int OP, int DK, int DV, int TV, int NT>
-__global__ void __launch_bounds__(NT, 65536 / (NT * 64))
+// The same step over a slot list, each slot at its own log length: list
+// entries [0, nfold) take the merge-token, the rest the append, in one
+// launch whatever the spread of lengths.  Blocks [0, nfold * H * DV / TVF)
+// are the merge-token units, on TVF-column tiles (8 rows a thread, the
+// logged value factors in registers for logs of up to LB entries); the rest
+// are the append units, on TVA-column tiles at the append's own shape (16
+// rows a thread where that leaves a thread per key row and value column).
+// One thread count NT serves both ranges.  The merge-token entries come
+// first, so that their longer CTAs start in the first wave rather than in
+// the tail.
+template <int OP, int DK, int DV, int TVA, int TVF, int NT, int LB>
+__global__ void __launch_bounds__(NT, 640 / NT)
 append_slots_kernel(const AppendParams p, const SlotList sl) {
-    using T = Tile<DK, DV, TV, NT>;
-    const int lh = (int)blockIdx.x / T::NVT, vt = (int)blockIdx.x - lh * T::NVT;
-    const int i = lh / p.H;
-    const int head = (int)sl.id[i] * p.H + (lh - i * p.H);
-    if (i < sl.nfold)
-        append_unit<OP, DK, DV, TV, NT, true, 0>(p, head, vt, sl.L[i]);
-    else
-        append_unit<OP, DK, DV, TV, NT, false, 0>(p, head, vt, sl.L[i]);
+    const int fold_units = sl.nfold * p.H * (DV / TVF);
+    int b = (int)blockIdx.x;
+    if (b < fold_units) {
+        constexpr int NVT = DV / TVF;
+        const int lh = b / NVT, i = lh / p.H;
+        merge_token_unit<OP, DK, DV, TVF, NT, LB>(p, (int)sl.id[i] * p.H + (lh - i * p.H), b - lh * NVT,
+                                                  sl.L[i]);
+    } else {
+        b -= fold_units;
+        constexpr int NVT = DV / TVA;
+        const int lh = b / NVT + sl.nfold * p.H, i = lh / p.H;
+        append_unit<OP, DK, DV, TVA, NT>(p, (int)sl.id[i] * p.H + (lh - i * p.H), b - (b / NVT) * NVT,
+                                         sl.L[i]);
+    }
 }
 
 // ================================================= merge / materialise ==

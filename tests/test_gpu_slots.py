@@ -97,7 +97,7 @@ def _compare(w, outs, o_ref, act):
 
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (128, 64)])
-@pytest.mark.parametrize("C", [1, 3, 4, 8])
+@pytest.mark.parametrize("C", [1, 3, 4, 8, 16])
 @pytest.mark.parametrize("mode", MODES)
 def test_slots_match_oracle(op, dims, C, mode):
     T = 3 * C + 5
