@@ -533,10 +533,15 @@ def measure(w, R, args, dev, stream, peaks, headline):
         cyc_st = B.Cycle([L_.handle for L_ in stag], _ios(w, xs, outs, R, C))
         ms = _time_graph(lambda: cyc_st.launch(stream), stream, args.steps, args.warmup, dev)
         ms, _ = reduce_over_ranks(ms / args.steps, 0, dev)
+        # each token of each layer is one slot-list launch: time them alone
+        kd_st = kernel_durations(stag, xs, outs, w, R, C, stream, dev, reps=3,
+                                 prime=lambda: cyc_st.launch(stream))
+        slot_us = statistics.mean([x for v in kd_st.values() for x in v]) * 1e3
         res["staggered"] = {
             "us_per_token": ms * 1e3 / (C * R),
             "hbm_gbs": gbs * us_per_token / (ms * 1e3 / (C * R)),
             "kernels_per_step": cyc_st.kernels,
+            "slot_kernel_us": slot_us,
             "slot_lengths": "slot b at b mod C when the cycle starts"}
         cyc_st.close()
         del stag
