@@ -40,12 +40,12 @@ cudaError_t launch_kernel(Kernel kern, unsigned grid, int threads, size_t smem, 
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int OP, int DK, int DV, int TV, bool FOLD, int LB>
+template <int OP, int DK, int DV, int TV, bool FOLD, int LB, int LX = -1>
 cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = AppendShape<DK, TV, FOLD>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     static std::atomic<int> resident[64];
-    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB>;
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB, LX>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
     const size_t smem_max = op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes;
@@ -67,10 +67,20 @@ cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
 
 // The merge-token keeps the logged value factors in registers while the log
 // is short; longer logs are read from shared memory.  The merge-token sees
-// L = C - 1, so the buckets end at 3 and 7 (C = 4 and C = 8 without padding).
+// L = C - 1, so the buckets end at 3 and 7 (C = 4 and C = 8 without padding),
+// and the log lengths of C = 4 and 8 have kernels of their own (measured on
+// B200, merge-token GDN C8 61.3 -> 54.6 us, KDA C8 117 -> 104 us).  A kernel
+// of its own for L = 1 (C = 2) is not built: its first launch raised "an
+// illegal instruction was encountered" in two of four runs, for a cause not
+// found in its source.
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     if constexpr (FOLD) {
+        switch (p.L) {
+            case 3: return launch_lb<OP, DK, DV, TV, true, 3, 3>(p, s);
+            case 7: return launch_lb<OP, DK, DV, TV, true, 7, 7>(p, s);
+            default: break;
+        }
         if (p.L <= 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
         if (p.L <= 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
     }
@@ -93,13 +103,13 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
 // entries (the first sl.nfold) are all at that length, one short of full.
 // Merge-token units use 32-column tiles, so that the thread count of the
 // append's shape gives them 8 rows a thread.
-template <int OP, int DK, int DV, int TVA, int LB>
+template <int OP, int DK, int DV, int TVA, int LB, int LX = -1>
 cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
     constexpr int TVF = 32;
     constexpr int NT = AppendShape<DK, TVA, false>::NT;
     static_assert(TVF <= NT && DK <= NT && (DK / (NT / (TVF / 4))) == 8, "merge-token tile shape");
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = append_slots_kernel<OP, DK, DV, TVA, TVF, NT, LB>;
+    auto kern = append_slots_kernel<OP, DK, DV, TVA, TVF, NT, LB, LX>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t sa = op_layout<OP, DK, TVA>(p.L, ie, true, false).bytes;
     const size_t sf = op_layout<OP, DK, TVF>(p.L, ie, true, true).bytes;
@@ -114,6 +124,13 @@ cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStrea
 
 template <int OP, int DK, int DV, int TVA>
 cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+    if (sl.nfold > 0) {
+        switch (p.L) {            // the merge-token entries' length, as in launch_tv
+            case 3: return launch_slots_lb<OP, DK, DV, TVA, 3, 3>(p, sl, s);
+            case 7: return launch_slots_lb<OP, DK, DV, TVA, 7, 7>(p, sl, s);
+            default: break;
+        }
+    }
     if (sl.nfold > 0 && p.L <= 3) return launch_slots_lb<OP, DK, DV, TVA, 3>(p, sl, s);
     if (sl.nfold > 0 && p.L <= 7) return launch_slots_lb<OP, DK, DV, TVA, 7>(p, sl, s);
     return launch_slots_lb<OP, DK, DV, TVA, 0>(p, sl, s);

@@ -744,10 +744,14 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
 //            o = scale (x_q + (k.q) u),  S_t = S' + k u^T
 //   RWKV6    o = scale (S'^T r + (r.(bonus*k)) v),  S_t = D(e^{g_t}) S' + k v^T
 // LB > 0 keeps the L <= LB logged value factors of the thread's columns in
-// registers; LB = 0 reads them from shared memory per row.
-template <int OP, int DK, int DV, int TV, int NT, int LB>
+// registers; LB = 0 reads them from shared memory per row.  LX >= 0 fixes
+// the log length at compile time (L = LX, the common capacities), so that
+// the table and fold loops have constant trip counts.
+template <int OP, int DK, int DV, int TV, int NT, int LB, int LX = -1>
 __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const int head, const int vt,
-                                                 const int L) {
+                                                 const int Lrt) {
+    static_assert(LX < 0 || LX <= LB, "a fixed log length must fit the register bucket");
+    const int L = LX >= 0 ? LX : Lrt;
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
     constexpr int NA = (OP == OP_RWKV6) ? 1 : 2;
@@ -797,6 +801,7 @@ __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const in
 
     // 3. replay-factor table A[i][j] = e^{Lambda_r[i] - Lambda_j[i]} k_j[i],
     //    base decay, read-out weights (all threads); the self term (warp 0)
+#pragma unroll
     for (int idx = tid; idx < DK * (L + 1); idx += NT) {
         const int i = idx % DK, j = idx / DK;
         const int x = (OP == OP_GDN) ? 0 : i;
@@ -889,8 +894,8 @@ __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const in
     }
 }
 
-template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0>
-__global__ void __launch_bounds__(NT)
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0, int LX = -1>
+__global__ void __launch_bounds__(NT, FOLD ? 768 / NT : 640 / NT)
 append_kernel(const AppendParams p, const Stagger st) {
     using T = Tile<DK, DV, TV, NT>;
     // The first wave's CTAs of an SM would otherwise run their serial phases
@@ -900,7 +905,7 @@ append_kernel(const AppendParams p, const Stagger st) {
         __nanosleep((unsigned)((int)blockIdx.x / st.sms) * (unsigned)st.ns);
     const int lh = (int)blockIdx.x / T::NVT;
     if constexpr (FOLD)
-        merge_token_unit<OP, DK, DV, TV, NT, LB>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
+        merge_token_unit<OP, DK, DV, TV, NT, LB, LX>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
     else
         append_unit<OP, DK, DV, TV, NT>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
 }
@@ -921,7 +926,7 @@ append_kernel(const AppendParams p, const Stagger st) {
 // the slots at staggered lengths, spread vs first: GDN d128 C8 27.2 vs
 // 28.8 us/token, KDA d128 C8 53.2 vs 57.3, RWKV6 d64 C8 17.2 vs 16.0, RWKV6
 // d64 C4 16.8 vs 17.0.
-template <int OP, int DK, int DV, int TVA, int TVF, int NT, int LB>
+template <int OP, int DK, int DV, int TVA, int TVF, int NT, int LB, int LX = -1>
 __global__ void __launch_bounds__(NT, 640 / NT)
 append_slots_kernel(const AppendParams p, const SlotList sl) {
     constexpr bool SPREAD = DK > 64;
@@ -932,8 +937,8 @@ append_slots_kernel(const AppendParams p, const SlotList sl) {
     if (SPREAD ? (b + 1) * F / N > f0 : b < F) {
         constexpr int NVT = DV / TVF;
         const int u = (int)f0, lh = u / NVT, i = lh / p.H;
-        merge_token_unit<OP, DK, DV, TVF, NT, LB>(p, (int)sl.id[i] * p.H + (lh - i * p.H), u - lh * NVT,
-                                                  sl.L[i]);
+        merge_token_unit<OP, DK, DV, TVF, NT, LB, LX>(p, (int)sl.id[i] * p.H + (lh - i * p.H), u - lh * NVT,
+                                                      sl.L[i]);
     } else {
         constexpr int NVT = DV / TVA;
         const int u = (int)(b - f0), lh = u / NVT + sl.nfold * p.H, i = lh / p.H;
