@@ -40,12 +40,12 @@ cudaError_t launch_kernel(Kernel kern, unsigned grid, int threads, size_t smem, 
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int OP, int DK, int DV, int TV, bool FOLD, int LB, int LX = -1>
+template <int OP, int DK, int DV, int TV, bool FOLD, int LX = -1>
 cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = AppendShape<DK, TV, FOLD>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     static std::atomic<int> resident[64];
-    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LB, LX>;
+    auto kern = append_kernel<OP, DK, DV, TV, NT, FOLD, LX>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, true, FOLD).bytes;
     const size_t smem_max = op_layout<OP, DK, TV>(MAXC - 1, 4, true, FOLD).bytes;
@@ -65,26 +65,19 @@ cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
     return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p, st);
 }
 
-// The merge-token keeps the logged value factors in registers while the log
-// is short; longer logs are read from shared memory.  The merge-token sees
-// L = C - 1, so the buckets end at 3 and 7 (C = 4 and C = 8 without padding),
-// and the log lengths of C = 4 and 8 have kernels of their own (measured on
-// B200, merge-token GDN C8 61.3 -> 54.6 us, KDA C8 117 -> 104 us).  A kernel
-// of its own for L = 1 (C = 2) is not built: its first launch raised "an
-// illegal instruction was encountered" in two of four runs, for a cause not
-// found in its source.
+// The merge-token sees L = C - 1: the log lengths of C = 4 and 8 have
+// kernels of their own (measured on B200: merge-token GDN C8 61.3 -> 54.6
+// us, KDA C8 117 -> 104 us), the others take the length at run time.  A
+// kernel of its own for L = 1 (C = 2) is not built: its first launch raised
+// "an illegal instruction was encountered" in two of four runs, for a cause
+// not found in its source.
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     if constexpr (FOLD) {
-        switch (p.L) {
-            case 3: return launch_lb<OP, DK, DV, TV, true, 3, 3>(p, s);
-            case 7: return launch_lb<OP, DK, DV, TV, true, 7, 7>(p, s);
-            default: break;
-        }
-        if (p.L <= 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
-        if (p.L <= 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
+        if (p.L == 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
+        if (p.L == 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
     }
-    return launch_lb<OP, DK, DV, TV, FOLD, 0>(p, s);
+    return launch_lb<OP, DK, DV, TV, FOLD>(p, s);
 }
 
 template <int OP, int DK, int DV, bool FOLD>
@@ -101,15 +94,18 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
 
 // Slot list: p.L is the longest length in the list; the merge-token
 // entries (the first sl.nfold) are all at that length, one short of full.
-// Merge-token units use 32-column tiles, so that the thread count of the
-// append's shape gives them 8 rows a thread.
-template <int OP, int DK, int DV, int TVA, int LB, int LX = -1>
+// For d_k = 128 the merge-token units take 32-column tiles (8 rows a thread
+// at the append's thread count), for d_k = 64 the append's own tile.
+// Measured on B200, cycles with the slots at staggered lengths, 32-column vs
+// the append's tile: GDN d128 C8 26.1 vs 28.7 us/token, KDA d128 C8 52.0 vs
+// 55.7; RWKV6 d64 C8 15.7 vs 14.4, C4 16.3 vs 15.6.
+template <int OP, int DK, int DV, int TVA, int LX = -1>
 cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
-    constexpr int TVF = 32;
+    constexpr int TVF = DK > 64 ? 32 : TVA;
     constexpr int NT = AppendShape<DK, TVA, false>::NT;
-    static_assert(TVF <= NT && DK <= NT && (DK / (NT / (TVF / 4))) == 8, "merge-token tile shape");
+    static_assert(TVF <= NT && DK <= NT, "merge-token tile shape");
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = append_slots_kernel<OP, DK, DV, TVA, TVF, NT, LB, LX>;
+    auto kern = append_slots_kernel<OP, DK, DV, TVA, TVF, NT, LX>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t sa = op_layout<OP, DK, TVA>(p.L, ie, true, false).bytes;
     const size_t sf = op_layout<OP, DK, TVF>(p.L, ie, true, true).bytes;
@@ -124,16 +120,10 @@ cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStrea
 
 template <int OP, int DK, int DV, int TVA>
 cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
-    if (sl.nfold > 0) {
-        switch (p.L) {            // the merge-token entries' length, as in launch_tv
-            case 3: return launch_slots_lb<OP, DK, DV, TVA, 3, 3>(p, sl, s);
-            case 7: return launch_slots_lb<OP, DK, DV, TVA, 7, 7>(p, sl, s);
-            default: break;
-        }
-    }
-    if (sl.nfold > 0 && p.L <= 3) return launch_slots_lb<OP, DK, DV, TVA, 3>(p, sl, s);
-    if (sl.nfold > 0 && p.L <= 7) return launch_slots_lb<OP, DK, DV, TVA, 7>(p, sl, s);
-    return launch_slots_lb<OP, DK, DV, TVA, 0>(p, sl, s);
+    // the merge-token entries' length is p.L: kernels of their own as in launch_tv
+    if (sl.nfold > 0 && p.L == 3) return launch_slots_lb<OP, DK, DV, TVA, 3>(p, sl, s);
+    if (sl.nfold > 0 && p.L == 7) return launch_slots_lb<OP, DK, DV, TVA, 7>(p, sl, s);
+    return launch_slots_lb<OP, DK, DV, TVA>(p, sl, s);
 }
 
 template <int OP, int DK, int DV>

@@ -11,9 +11,9 @@
 // there are too few heads to fill the GPU (the paper's value-tile split): TV
 // value columns of all d_k rows, so the key-side contractions S^T x reduce
 // inside the CTA.  TV/4 threads per row, each owning a 16-byte column group,
-// and RPT rows per thread held in registers: 16 for the append, 8 for the
-// merge-token, merge and eager kernels (the launchers pick NT; Tile derives
-// the rest).  The eager kernel always uses 32-column tiles.  Nothing here is
+// and RPT rows per thread held in registers: 16 for the append and the
+// merge-token, 8 for the merge and eager kernels (the launchers pick NT;
+// Tile derives the rest).  The eager kernel always uses 32-column tiles.  Nothing here is
 // a dense contraction worth a tensor core: per state element the append does
 // 2 FMAs and the merge at most C = 16, against 4 to 8 bytes of HBM traffic.
 #pragma once
@@ -743,14 +743,11 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
 //   GDN/KDA  x_k = S'^T k, x_q = S'^T q, u = beta (v - x_k),
 //            o = scale (x_q + (k.q) u),  S_t = S' + k u^T
 //   RWKV6    o = scale (S'^T r + (r.(bonus*k)) v),  S_t = D(e^{g_t}) S' + k v^T
-// LB > 0 keeps the L <= LB logged value factors of the thread's columns in
-// registers; LB = 0 reads them from shared memory per row.  LX >= 0 fixes
-// the log length at compile time (L = LX, the common capacities), so that
-// the table and fold loops have constant trip counts.
-template <int OP, int DK, int DV, int TV, int NT, int LB, int LX = -1>
+// LX >= 0 fixes the log length at compile time (L = LX, the common
+// capacities), so that the table and fold loops have constant trip counts.
+template <int OP, int DK, int DV, int TV, int NT, int LX = -1>
 __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const int head, const int vt,
                                                  const int Lrt) {
-    static_assert(LX < 0 || LX <= LB, "a fixed log length must fit the register bucket");
     const int L = LX >= 0 ? LX : Lrt;
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
@@ -832,26 +829,38 @@ __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const in
     }
     __syncthreads();
 
-    // 4. fold the log into the tile, then (a second pass, so that the logged
-    //    factors and the accumulators are not live together) read out
-    //    x_a[c] = sum_i w_a[i] S'[i][c]
+    // 4. fold the log into the tile, four logged entries at a time (their
+    //    value factors for the thread's columns in registers, the rows swept
+    //    once per four entries), then read out x_a[c] = sum_i w_a[i] S'[i][c]
+    //    in a pass of its own, so that factors and accumulators are not live
+    //    together
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-    if constexpr (LB > 0) {
-        float4 ur[LB];
 #pragma unroll
-        for (int j = 0; j < LB; ++j)
-            ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < T::RPT; ++r) {
+        const float g = s_gam[rg + r * T::RG];
+        const float2 g2 = make_float2(g, g);
+        const float2 lo = __fmul2_rn(g2, make_float2(s[r].x, s[r].y)), hi = __fmul2_rn(g2, make_float2(s[r].z, s[r].w));
+        s[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    auto fold_chunk = [&](const int j0) {
+        float4 ur[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            ur[jj] = (j0 + jj < L) ? ld_raw4(dsm + lay.U, (j0 + jj) * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            s[r] = fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L);
+            const float4 cf4 = *reinterpret_cast<const float4 *>(A + (rg + r * T::RG) * AP + j0);
+            const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                if (j0 + jj < L) fma4(s[r], cf[jj], ur[jj]);
         }
+    };
+    if constexpr (LX >= 0) {
+#pragma unroll
+        for (int j0 = 0; j0 < LX; j0 += 4) fold_chunk(j0);
     } else {
-#pragma unroll
-        for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            s[r] = fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf);
-        }
+        for (int j0 = 0; j0 < L; j0 += 4) fold_chunk(j0);
     }
     float xc[NA];
     {
@@ -894,8 +903,8 @@ __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const in
     }
 }
 
-template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LB = 0, int LX = -1>
-__global__ void __launch_bounds__(NT, FOLD ? 768 / NT : 640 / NT)
+template <int OP, int DK, int DV, int TV, int NT, bool FOLD, int LX = -1>
+__global__ void __launch_bounds__(NT, 640 / NT)
 append_kernel(const AppendParams p, const Stagger st) {
     using T = Tile<DK, DV, TV, NT>;
     // The first wave's CTAs of an SM would otherwise run their serial phases
@@ -905,20 +914,20 @@ append_kernel(const AppendParams p, const Stagger st) {
         __nanosleep((unsigned)((int)blockIdx.x / st.sms) * (unsigned)st.ns);
     const int lh = (int)blockIdx.x / T::NVT;
     if constexpr (FOLD)
-        merge_token_unit<OP, DK, DV, TV, NT, LB, LX>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
+        merge_token_unit<OP, DK, DV, TV, NT, LX>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
     else
         append_unit<OP, DK, DV, TV, NT>(p, lh, (int)blockIdx.x - lh * T::NVT, p.L);
 }
 
 // The same step over a slot list, each slot at its own log length: list
 // entries [0, nfold) take the merge-token, the rest the append, in one
-// launch whatever the spread of lengths.  The merge-token units run on
-// TVF-column tiles (8 rows a thread, the logged value factors in registers
-// for logs of up to LB entries), the append units on TVA-column tiles at the
-// append's own shape (16 rows a thread where that leaves a thread per key
-// row and value column); one thread count NT serves both.  For d_k = 128 a
-// merge-token unit moves about as many bytes per CTA lifetime as an append
-// unit (half the tile, read and written), and the two kinds are spread
+// launch whatever the spread of lengths.  The append units run on
+// TVA-column tiles at the append's own shape (16 rows a thread where that
+// leaves a thread per key row and value column), the merge-token units on
+// TVF-column tiles at the same thread count NT (the launcher picks TVF).
+// For d_k = 128 (TVF = 32, half the append's tile) a merge-token unit moves
+// about as many bytes per CTA lifetime as an append unit (half the tile,
+// read and written), and the two kinds are spread
 // evenly over the grid: block b is merge-token unit floor(b F / N) when that
 // count steps at b (F merge-token units of N), else append unit
 // b - floor(b F / N), so every wave keeps the launch's mix in flight.  For
@@ -926,7 +935,7 @@ append_kernel(const AppendParams p, const Stagger st) {
 // the slots at staggered lengths, spread vs first: GDN d128 C8 27.2 vs
 // 28.8 us/token, KDA d128 C8 53.2 vs 57.3, RWKV6 d64 C8 17.2 vs 16.0, RWKV6
 // d64 C4 16.8 vs 17.0.
-template <int OP, int DK, int DV, int TVA, int TVF, int NT, int LB, int LX = -1>
+template <int OP, int DK, int DV, int TVA, int TVF, int NT, int LX = -1>
 __global__ void __launch_bounds__(NT, 640 / NT)
 append_slots_kernel(const AppendParams p, const SlotList sl) {
     constexpr bool SPREAD = DK > 64;
@@ -937,7 +946,7 @@ append_slots_kernel(const AppendParams p, const SlotList sl) {
     if (SPREAD ? (b + 1) * F / N > f0 : b < F) {
         constexpr int NVT = DV / TVF;
         const int u = (int)f0, lh = u / NVT, i = lh / p.H;
-        merge_token_unit<OP, DK, DV, TVF, NT, LB, LX>(p, (int)sl.id[i] * p.H + (lh - i * p.H), u - lh * NVT,
+        merge_token_unit<OP, DK, DV, TVF, NT, LX>(p, (int)sl.id[i] * p.H + (lh - i * p.H), u - lh * NVT,
                                                       sl.L[i]);
     } else {
         constexpr int NVT = DV / TVA;

@@ -49,16 +49,19 @@ struct CtaShape {
     static constexpr int NT = (TV / 4) * (DK / 8);
 };
 
-// The append (not the merge-token, which also holds the logged value factors
-// in registers) streams 16 rows per thread where that still leaves a thread
-// per key row and per value column: 96 registers a thread, so 5 CTAs of 128
-// threads fit an SM and 160 KB of the base is in flight per SM instead of
-// 128 KB.  Measured on B200 in four-layer merge cycles against 8 rows per
-// thread: GDN -4.2 %, KDA -4.9 %, RWKV6 (d = 64) -0.3 % per token.
+// The append and the merge-token stream 16 rows per thread where that still
+// leaves a thread per key row and per value column: at most 96 registers a
+// thread, so 5 CTAs of 128 threads fit an SM and 160 KB of the base is in
+// flight per SM instead of 128 KB (the merge-token folds its log four
+// entries at a time, so that only four value factors a thread are held in
+// registers).  Measured on B200 in four-layer merge cycles against 8 rows per
+// thread: append GDN -4.2 %, KDA -4.9 %, RWKV6 (d = 64) -0.3 % per token;
+// merge-token GDN C8 53.3 -> 48.8 us, KDA C8 99.3 -> 91.9 us (cycles GDN
+// -0.8 %, KDA -1.2 %, RWKV6 C4 -3.8 %, RWKV6 C8 +1.4 %).
 template <int DK, int TV, bool FOLD>
 struct AppendShape {
     static constexpr int NT16 = (TV / 4) * (DK / 16);
-    static constexpr int NT = (!FOLD && NT16 >= (DK > TV ? DK : TV)) ? NT16 : CtaShape<DK, TV>::NT;
+    static constexpr int NT = (NT16 >= (DK > TV ? DK : TV)) ? NT16 : CtaShape<DK, TV>::NT;
 };
 
 // Raise a kernel's dynamic shared-memory limit once per device.
