@@ -508,47 +508,6 @@ __device__ __forceinline__ void replay_table(float *A, float *gam, const float *
     }
 }
 
-// New state row segment: gam * s + sum_{j<L} A[row][j] U_j[c4..c4+3] (+ kr * w4)
-template <int TV>
-__device__ __forceinline__ float4 fold_row(float4 s, float gm, const float *Arow, const unsigned char *sU,
-                                           int c4, int L, int ubf) {
-    const float2 g2 = make_float2(gm, gm);
-    const float2 olo = __fmul2_rn(g2, make_float2(s.x, s.y)), ohi = __fmul2_rn(g2, make_float2(s.z, s.w));
-    float4 o = make_float4(olo.x, olo.y, ohi.x, ohi.y);
-    for (int j0 = 0; j0 < L; j0 += 4) {
-        const float4 cf4 = *reinterpret_cast<const float4 *>(Arow + j0);
-        const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            if (j0 + jj < L) {
-                fma4(o, cf[jj], ld_raw4(sU, (j0 + jj) * TV + c4, ubf));
-            }
-        }
-    }
-    return o;
-}
-
-// The same with the L <= LB value factors of this thread's four columns held
-// in registers (loaded once, reused for every row of the tile).
-template <int LB>
-__device__ __forceinline__ float4 fold_row_reg(float4 s, float gm, const float *Arow,
-                                               const float4 (&ur)[LB], int L) {
-    const float2 g2 = make_float2(gm, gm);
-    const float2 olo = __fmul2_rn(g2, make_float2(s.x, s.y)), ohi = __fmul2_rn(g2, make_float2(s.z, s.w));
-    float4 o = make_float4(olo.x, olo.y, ohi.x, ohi.y);
-#pragma unroll
-    for (int j0 = 0; j0 < LB; j0 += 4) {
-        if (j0 < L) {
-            const float4 cf4 = *reinterpret_cast<const float4 *>(Arow + j0);
-            const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                if (j0 + jj < LB && j0 + jj < L) fma4(o, cf[jj], ur[j0 + jj]);
-        }
-    }
-    return o;
-}
-
 // ============================================ append + read-out (+ fold) ==
 //
 // One CTA per unit (a head, or a TV-column value tile of a head).
@@ -962,9 +921,12 @@ append_slots_kernel(const AppendParams p, const SlotList sl) {
 // (Lambda_L = the last entry's snapshot; L = 0 copies the base).  In place
 // (dst == base) it is the merge; into another buffer it is materialise.
 // One CTA per unit; the register tile is loaded first, the log staged by
-// warp 0, the replay-factor table built once per CTA.
-template <int OP, int DK, int DV, int TV, int NT, int LB = 0, bool SLOTS = false>
-__global__ void __launch_bounds__(NT)
+// warp 0, the replay-factor table built once per CTA, and the log folded
+// into the tile four entries at a time as in the merge-token (the four value
+// factors of the thread's columns in registers, each row's four
+// coefficients one 16-byte shared load).
+template <int OP, int DK, int DV, int TV, int NT, bool SLOTS = false>
+__global__ void __launch_bounds__(NT, 640 / NT)
 merge_kernel(const MergeParams p, const SlotArg<SLOTS> sl) {
     using T = Tile<DK, DV, TV, NT>;
     constexpr int M = (OP == OP_GDN) ? 1 : DK;
@@ -1005,25 +967,29 @@ merge_kernel(const MergeParams p, const SlotArg<SLOTS> sl) {
     const float *A = reinterpret_cast<const float *>(dsm + lay.A);
     const int AP = up4(L) + 4;
     const int ubf = (OP == OP_RWKV6) ? p.in_bf16 : 0;
-    if constexpr (LB > 0) {
-        // the logged value factors of this thread's columns, once
-        float4 ur[LB];
 #pragma unroll
-        for (int j = 0; j < LB; ++j)
-            ur[j] = (j < L) ? ld_raw4(dsm + lay.U, j * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < T::RPT; ++r) {
+        const float g = s_gam[rg + r * T::RG];
+        const float2 g2 = make_float2(g, g);
+        const float2 lo = __fmul2_rn(g2, make_float2(s[r].x, s[r].y)), hi = __fmul2_rn(g2, make_float2(s[r].z, s[r].w));
+        s[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    for (int j0 = 0; j0 < L; j0 += 4) {
+        float4 ur[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            ur[jj] = (j0 + jj < L) ? ld_raw4(dsm + lay.U, (j0 + jj) * TV + c4, ubf) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            st_state(dh + (size_t)row * DV, fold_row_reg<LB>(s[r], s_gam[row], A + row * AP, ur, L));
-        }
-    } else {
+            const float4 cf4 = *reinterpret_cast<const float4 *>(A + (rg + r * T::RG) * AP + j0);
+            const float cf[4] = {cf4.x, cf4.y, cf4.z, cf4.w};
 #pragma unroll
-        for (int r = 0; r < T::RPT; ++r) {
-            const int row = rg + r * T::RG;
-            st_state(dh + (size_t)row * DV,
-                     fold_row<TV>(s[r], s_gam[row], A + row * AP, dsm + lay.U, c4, L, ubf));
+            for (int jj = 0; jj < 4; ++jj)
+                if (j0 + jj < L) fma4(s[r], cf[jj], ur[jj]);
         }
     }
+#pragma unroll
+    for (int r = 0; r < T::RPT; ++r) st_state(dh + (size_t)(rg + r * T::RG) * DV, s[r]);
 }
 
 // ================================================================ eager ==

@@ -17,11 +17,14 @@ long long launch_heads(const MergeParams &p, const SlotArg<SLOTS> &sl) {
 }
 
 // p.L is the shared length, or for a slot list the longest length in it.
-template <int OP, int DK, int DV, int TV, int LB, bool SLOTS>
-cudaError_t launch_lb(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
-    constexpr int NT = CtaShape<DK, TV>::NT;
+// The thread count is the append's: 16 rows a thread where that leaves a
+// thread per key row and value column (at most 96 registers, 5 CTAs of 128
+// threads per SM).
+template <int OP, int DK, int DV, int TV, bool SLOTS>
+cudaError_t launch_tv(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
+    constexpr int NT = AppendShape<DK, TV, true>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
-    auto kern = merge_kernel<OP, DK, DV, TV, NT, LB, SLOTS>;
+    auto kern = merge_kernel<OP, DK, DV, TV, NT, SLOTS>;
     const int ie = p.in_bf16 ? 2 : 4;
     const size_t smem = op_layout<OP, DK, TV>(p.L, ie, false, true).bytes;
     cudaError_t e = allow_smem(smem_ok, kern, op_layout<OP, DK, TV>(MAXC, 4, false, true).bytes);
@@ -29,14 +32,6 @@ cudaError_t launch_lb(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream
     const unsigned grid = (unsigned)(launch_heads<SLOTS>(p, sl) * (DV / TV));
     kern<<<grid, NT, smem, s>>>(p, sl);
     return cudaGetLastError();
-}
-
-// The logged value factors stay in registers for logs of up to 8 entries.
-template <int OP, int DK, int DV, int TV, bool SLOTS>
-cudaError_t launch_tv(const MergeParams &p, const SlotArg<SLOTS> &sl, cudaStream_t s) {
-    if (p.L <= 4) return launch_lb<OP, DK, DV, TV, 4, SLOTS>(p, sl, s);
-    if (p.L <= 8) return launch_lb<OP, DK, DV, TV, 8, SLOTS>(p, sl, s);
-    return launch_lb<OP, DK, DV, TV, 0, SLOTS>(p, sl, s);
 }
 
 template <int OP, int DK, int DV, bool SLOTS>
