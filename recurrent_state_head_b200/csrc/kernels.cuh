@@ -11,8 +11,8 @@
 // there are too few heads to fill the GPU (the paper's value-tile split): TV
 // value columns of all d_k rows, so the key-side contractions S^T x reduce
 // inside the CTA.  TV/4 threads per row, each owning a 16-byte column group,
-// and RPT rows per thread held in registers: 16 for the append and the
-// merge-token, 8 for the merge and eager kernels (the launchers pick NT;
+// and RPT rows per thread held in registers: 16 for the append, the
+// merge-token and the merge, 8 for the eager kernel (the launchers pick NT;
 // Tile derives the rest).  The eager kernel always uses 32-column tiles.  Nothing here is
 // a dense contraction worth a tensor core: per state element the append does
 // 2 FMAs and the merge at most C = 16, against 4 to 8 bytes of HBM traffic.
