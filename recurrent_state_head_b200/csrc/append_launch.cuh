@@ -41,7 +41,7 @@ cudaError_t launch_kernel(Kernel kern, unsigned grid, int threads, size_t smem, 
 }
 
 template <int OP, int DK, int DV, int TV, bool FOLD, int LX = -1>
-cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
+cudaError_t launch_one(const AppendParams &p, cudaStream_t s) {
     constexpr int NT = AppendShape<DK, TV, FOLD>::NT;
     static std::atomic<unsigned long long> smem_ok{0};
     static std::atomic<int> resident[64];
@@ -74,10 +74,10 @@ cudaError_t launch_lb(const AppendParams &p, cudaStream_t s) {
 template <int OP, int DK, int DV, int TV, bool FOLD>
 cudaError_t launch_tv(const AppendParams &p, cudaStream_t s) {
     if constexpr (FOLD) {
-        if (p.L == 3) return launch_lb<OP, DK, DV, TV, true, 3>(p, s);
-        if (p.L == 7) return launch_lb<OP, DK, DV, TV, true, 7>(p, s);
+        if (p.L == 3) return launch_one<OP, DK, DV, TV, true, 3>(p, s);
+        if (p.L == 7) return launch_one<OP, DK, DV, TV, true, 7>(p, s);
     }
-    return launch_lb<OP, DK, DV, TV, FOLD>(p, s);
+    return launch_one<OP, DK, DV, TV, FOLD>(p, s);
 }
 
 template <int OP, int DK, int DV, bool FOLD>
@@ -100,7 +100,7 @@ cudaError_t launch_fold(const AppendParams &p, cudaStream_t s) {
 // the append's tile: GDN d128 C8 26.1 vs 28.7 us/token, KDA d128 C8 52.0 vs
 // 55.7; RWKV6 d64 C8 15.7 vs 14.4, C4 16.3 vs 15.6.
 template <int OP, int DK, int DV, int TVA, int LX = -1>
-cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
+cudaError_t launch_slots_one(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
     constexpr int TVF = DK > 64 ? 32 : TVA;
     constexpr int NT = AppendShape<DK, TVA, false>::NT;
     static_assert(TVF <= NT && DK <= NT, "merge-token tile shape");
@@ -121,9 +121,9 @@ cudaError_t launch_slots_lb(const AppendParams &p, const SlotList &sl, cudaStrea
 template <int OP, int DK, int DV, int TVA>
 cudaError_t launch_slots_tv(const AppendParams &p, const SlotList &sl, cudaStream_t s) {
     // the merge-token entries' length is p.L: kernels of their own as in launch_tv
-    if (sl.nfold > 0 && p.L == 3) return launch_slots_lb<OP, DK, DV, TVA, 3>(p, sl, s);
-    if (sl.nfold > 0 && p.L == 7) return launch_slots_lb<OP, DK, DV, TVA, 7>(p, sl, s);
-    return launch_slots_lb<OP, DK, DV, TVA>(p, sl, s);
+    if (sl.nfold > 0 && p.L == 3) return launch_slots_one<OP, DK, DV, TVA, 3>(p, sl, s);
+    if (sl.nfold > 0 && p.L == 7) return launch_slots_one<OP, DK, DV, TVA, 7>(p, sl, s);
+    return launch_slots_one<OP, DK, DV, TVA>(p, sl, s);
 }
 
 template <int OP, int DK, int DV>
