@@ -295,14 +295,13 @@ cudaError_t launch_slots(const dl_handle *h, bool merge, const std::vector<int> 
 dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active, const dl_step_io &io,
                       cudaStream_t st, bool early, int *kernels) {
     const int B = h->cfg.B, C = h->cfg.C, mode = h->cfg.auto_merge;
-    const char *full_msg = mode == DL_MERGE_OFF
-                               ? "log is full (L = C = %d) and auto_merge is off: merge first"
-                               : "log is full (L = C = %d) after a failed merge launch: call dl_merge";
+    const char *full_why = mode == DL_MERGE_OFF ? "auto_merge is off: merge first"
+                                                : "a merge failed to launch: call dl_merge";
     bool all = true;
     if (active)
         for (int b = 0; b < B && all; ++b) all = active[b] != 0;
     if (ln.shared && all) {
-        if (ln.L >= C) return fail(DL_ESTATE, full_msg, C);
+        if (ln.L >= C) return fail(DL_ESTATE, "log is full (L = C = %d); %s", C, full_why);
         if (mode == DL_MERGE_FOLD && ln.L == C - 1) {
             // the token that completes the log: one kernel reads the base once
             // and writes the merged logical state back
@@ -336,11 +335,7 @@ dl_status decode_step(const dl_handle *h, Lens &ln, const unsigned char *active,
         for (int b = 0; b < B; ++b) {
             if (active && !active[b]) continue;
             const int L = ln.of(b);
-            if (L >= C) {
-                char msg[160];
-                snprintf(msg, sizeof msg, "slot %d: %s", b, full_msg);
-                return fail(DL_ESTATE, msg, C);
-            }
+            if (L >= C) return fail(DL_ESTATE, "slot %d: log is full (L = C = %d); %s", b, C, full_why);
             const bool fold = mode == DL_MERGE_FOLD && L == C - 1;
             if (fold != (pass == 0)) continue;
             ids.push_back(b);
