@@ -54,3 +54,41 @@ def test_write_reduction_meets_half_capacity(name):
     assert ratio >= w.C / 2, (name, ratio)
     # the merge-token never writes more than the separate merge
     assert bm["token_write"] <= bench.bytes_model(w, fold=False)["token_write"]
+
+
+def test_config_object_and_l2_wording():
+    """Both arms print the same config object; a working set below the
+    126 MB L2 is labelled as such."""
+    big = synth.WORKLOADS["gdn-b128-h16-d128-c8"]
+    small = synth.WORKLOADS["gdn-b1-h2-d64-c4-fp32"]
+    cb = bench.workload_config(big, 4, 1)
+    assert cb["workload"] == big.name and cb["layers_rotated"] == 4
+    assert cb["l2"].startswith("inputs larger than L2")
+    assert "fits in L2" in bench.workload_config(small, 4, 1)["l2"]
+    assert set(cb) == set(bench.workload_config(small, 4, 1))
+
+
+@pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c4",
+                                  "rwkv6-b128-h32-d64-c8"])
+def test_device_drawn_timing_inputs(name):
+    """The sweep's device-drawn states and tokens have the workload's shapes,
+    dtypes and distributions (checked on the CPU generator)."""
+    import torch
+    from recurrent_state_head_b200 import device as D
+    w = synth.WORKLOADS[name].with_(B=4)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1)
+    S = D.draw_state(w, 0, "cpu", g)
+    assert S.shape == (w.heads, w.dk, w.dv) and S.dtype == torch.float32
+    assert abs(float(S.std()) - w.init_std) < 0.1 * w.init_std
+    x = D.draw_tokens(w, 3, "cpu", g)
+    assert x["q"].shape == (3, w.heads, w.dk) and x["v"].shape == (3, w.heads, w.dv)
+    assert x["g"].shape == (3, w.heads, w.m) and x["beta"].shape == (3, w.heads)
+    assert x["q"].dtype == D.TORCH_DTYPE[w.in_dtype]
+    assert bool((x["g"] < 0).all())
+    if w.op == synth.RWKV6:
+        assert bool((x["beta"] == 0).all())
+    else:
+        norms = x["k"].float().norm(dim=-1)
+        assert bool(((norms - 1).abs() < 1e-2).all())
+        assert bool(((x["beta"] > 0) & (x["beta"] < 1)).all())
