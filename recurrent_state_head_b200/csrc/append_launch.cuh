@@ -9,12 +9,13 @@
 namespace dl {
 namespace append_detail {
 
-// The first wave's CTAs of an SM start spread over kStaggerWindowNs (slot i
-// of n resident CTAs at i * window / n).  Measured on B200 in four-layer
-// merge cycles, append with four CTAs per SM, against no offset: GDN -2.3 %,
-// KDA -1.2 %, RWKV6 -2.5 % per token with 1.0 us between CTAs (0.6 us: the
-// same for GDN and KDA, -1 % for RWKV6; 1.5 us no better).
-constexpr int kStaggerWindowNs = 4000;
+// The first wave's CTAs of an SM start spread over a window (slot i of n
+// resident CTAs at i * window / n): 2 us for d_k = 128, 4 us for d_k = 64.
+// Measured on B200 in four-layer merge cycles, per token, 4 us against no
+// offset: GDN -2.3 %, KDA -1.3 %, RWKV6 -4.2 % (C = 8 and C = 4); 2 us
+// against 4 us: GDN -0.7 % (isolated append -1 %), KDA -0.2 %, RWKV6 +2.4 %.
+template <int DK>
+constexpr int stagger_window_ns() { return DK > 64 ? 2000 : 4000; }
 constexpr bool kStaggerFold = true;
 
 // Plain launch, or a programmatic dependent launch when p.early (it may
@@ -60,7 +61,7 @@ cudaError_t launch_one(const AppendParams &p, cudaStream_t s) {
         e = sm_count(&st.sms);
         if (e != cudaSuccess) return e;
         st.slots = slots;
-        st.ns = kStaggerWindowNs / slots;
+        st.ns = stagger_window_ns<DK>() / slots;
     }
     return launch_kernel(kern, grid, NT, smem, p.early != 0, s, p, st);
 }
