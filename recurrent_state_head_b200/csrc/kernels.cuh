@@ -524,7 +524,9 @@ __device__ __forceinline__ void replay_table(float *A, float *gam, const float *
 // append_kernel runs it (or merge_token_unit, below) over all heads at the
 // shared length p.L, and append_slots_kernel over a slot list whose first
 // nfold entries take the merge-token and the rest the append (one launch per
-// step however the slots' lengths are spread).
+// step however the slots' lengths are spread).  nap > 0 holds the unit for
+// nap nanoseconds once its base loads have gone out (a first-wave start
+// offset taken there; see append_kernel).
 template <int OP, int DK, int DV, int TV, int NT>
 __device__ __forceinline__ void append_unit(const AppendParams &p, const int head, const int vt,
                                             const int L, const unsigned nap = 0u) {
@@ -705,6 +707,7 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, const int hea
 //   RWKV6    o = scale (S'^T r + (r.(bonus*k)) v),  S_t = D(e^{g_t}) S' + k v^T
 // LX >= 0 fixes the log length at compile time (L = LX, the common
 // capacities), so that the table and fold loops have constant trip counts.
+// nap as for append_unit.
 template <int OP, int DK, int DV, int TV, int NT, int LX = -1>
 __device__ __forceinline__ void merge_token_unit(const AppendParams &p, const int head, const int vt,
                                                  const int Lrt, const unsigned nap = 0u) {
