@@ -48,6 +48,31 @@ MUTANTS = {
     "merge replays one entry too few":
         ("for (int j = 0; j < L; ++j) s += coef[j] * U[(size_t)j * dv + c];",
          "for (int j = 0; j + 1 < L; ++j) s += coef[j] * U[(size_t)j * dv + c];"),
+    "output scale dropped":
+        ("out[c] = scale * acc;", "out[c] = acc;"),
+    "replay reads the next snapshot":
+        ("Lam[(size_t)j * m + x]) * K[(size_t)j * dk + i]",
+         "Lam[(size_t)(j + 1 < L ? j + 1 : j) * m + x]) * K[(size_t)j * dk + i]"),
+    "base read-out decays to the previous snapshot":
+        ("double gam = exp(lam_t[didx(op, i)]);", "double gam = exp(lam_prev[didx(op, i)]);"),
+    "merge decays to the first snapshot":
+        ("double lamL = L > 0 ? Lam[(size_t)(L - 1) * m + x] : 0.0;",
+         "double lamL = L > 0 ? Lam[x] : 0.0;"),
+    "self term uses k.k":
+        ("kq += k[i] * q[i];", "kq += k[i] * k[i];"),
+    "rwkv6 bonus without the key":
+        ("rb += q[i] * bonus[i] * k[i];", "rb += q[i] * bonus[i];"),
+    "read-out with the key":
+        ("acc += S[(size_t)i * dv + c] * q[i];", "acc += S[(size_t)i * dv + c] * k[i];"),
+    "log stores the previous snapshot":
+        ("Lam[(size_t)L * m + x] = lam_t[x];", "Lam[(size_t)L * m + x] = lam_prev[x];"),
+    "log stores the query as key":
+        ("K[(size_t)L * dk + i] = k[i];", "K[(size_t)L * dk + i] = q[i];"),
+    "merge one token early":
+        ("if (L == C) {", "if (L == C - 1 || L == C) {"),
+    "rwkv6 read-out from the base without decay":
+        ("xr += base[(size_t)i * dv + c] * exp(lam_prev[i]) * q[i];",
+         "xr += base[(size_t)i * dv + c] * q[i];"),
 }
 
 PIN_CALLS = [
