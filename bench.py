@@ -126,14 +126,17 @@ _REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML on a thread."""
+    """Samples SM clock and clock-event reasons through NVML on a thread.
+    Entering waits (at most a second) for the thread's first sample, so
+    that a short timed region that follows is sampled from its start."""
 
-    def __init__(self, torch_device, period_s=0.005):
+    def __init__(self, torch_device, period_s=0.001):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
         self.h = None
         self._stop = threading.Event()
+        self._first = threading.Event()
         try:
             import pynvml as N
             N.nvmlInit()
@@ -163,12 +166,14 @@ class ClockSampler:
                                      int(fn(self.h))))
             except Exception:
                 pass
+            self._first.set()
             self._stop.wait(self.period)
 
     def __enter__(self):
         if self.h is not None:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
+            self._first.wait(1.0)
         return self
 
     def __exit__(self, *a):
