@@ -92,3 +92,60 @@ def test_device_drawn_timing_inputs(name):
         norms = x["k"].float().norm(dim=-1)
         assert bool(((norms - 1).abs() < 1e-2).all())
         assert bool(((x["beta"] > 0) & (x["beta"] < 1)).all())
+
+
+class _FakeNVML:
+    """Stands in for pynvml: a GPU whose (SM clock, clock-event reasons)
+    samples follow a script, the last entry repeating."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, script):
+        self.script = list(script)
+        self.calls = 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        return "h"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.script[min(self.calls, len(self.script) - 1)][0]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        r = self.script[min(self.calls, len(self.script) - 1)][1]
+        self.calls += 1
+        return r
+
+
+def test_clock_sampler_with_fake_nvml(monkeypatch):
+    """The sampler has its first sample before the timed region starts,
+    drops idle samples from the median and reports every reason seen."""
+    import sys
+    import time
+    import torch
+    fake = _FakeNVML([(345, 0x1)] + [(1800, 0x4)] * 4 + [(1965, 0x0)])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+
+    class Props:
+        uuid = "0000"
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: Props())
+
+    class Dev:
+        index = 0
+    with bench.ClockSampler(Dev(), period_s=0.001) as clk:
+        assert len(clk.samples) >= 1            # taken before the region
+        t0 = time.time()
+        while fake.calls < 16 and time.time() - t0 < 5:
+            time.sleep(0.002)
+    s = clk.summary()
+    assert s["sm_max_mhz"] == 1965
+    assert s["samples"] >= 10
+    assert s["sm_mhz"] == 1965                  # idle sample left out
+    assert s["reasons"] == ["sw_power_cap"]
