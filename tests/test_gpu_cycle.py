@@ -20,7 +20,8 @@ from recurrent_state_head_b200 import binding as B
 from recurrent_state_head_b200 import device as D
 from recurrent_state_head_b200 import synth
 
-from test_gpu_parity import MODES, OPS, TOL_STATE, oracle_inputs, small, to_np, tol_out
+from test_gpu_parity import (MODES, OPS, TOL_STATE, oracle_inputs, run_oracle_eager, small, to_np,
+                              tol_out)
 from test_gpu_slots import _oracle_materialize_slots, _oracle_slots
 
 pytestmark = pytest.mark.gpu
@@ -154,22 +155,25 @@ def test_cycle_staggered_with_empty_layer(op, mode, layout):
         assert [L_.slot_len(b) for b in range(w.B)] == Ltr[-1].tolist()
 
 
+@pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c8",
+                                  "rwkv6-b128-h32-d64-c8"])
 @pytest.mark.parametrize("mode", MODES)
-def test_cycle_full_size(mode):
-    """The GDN B128 H16 d128 C8 workload as a four-layer cycle (the bench's
-    step), two cycles: byte-for-byte equal to the same steps issued one by
-    one, and every head of every layer against the oracle (outputs of every
-    token, state after each cycle)."""
-    w = synth.WORKLOADS["gdn-b128-h16-d128-c8"]
+def test_cycle_full_size(mode, name):
+    """The bench's workloads as four-layer cycles (the bench's step), two
+    cycles: byte-for-byte equal to the same steps issued one by one, and
+    every head of every layer against the oracle (outputs of every token,
+    state after each cycle)."""
+    w = synth.WORKLOADS[name]
     C, R = w.C, 4
     T = 2 * C
-    a, b, xs, tis, S0s = [], [], [], [], []
+    a, b, xs, tis, S0s, bons = [], [], [], [], [], []
     for l in range(R):
         S0s.append(synth.initial_state(w, layer=l))
+        bons.append(synth.bonus(w, layer=l))
         tis.append(synth.tokens(w, 0, T, layer=l, want64=False))
         xs.append(D.to_device(tis[l], w))
-        a.append(D.DecodeLayer(w, S0s[l], None, auto_merge=mode))
-        b.append(D.DecodeLayer(w, S0s[l], None, auto_merge=mode))
+        a.append(D.DecodeLayer(w, S0s[l], bons[l], auto_merge=mode))
+        b.append(D.DecodeLayer(w, S0s[l], bons[l], auto_merge=mode))
     outs_a = [L_.new_out(T) for L_ in a]
     states_a, states_b = [], []
     for c in range(2):
@@ -183,14 +187,14 @@ def test_cycle_full_size(mode):
         assert torch.equal(outs_a[l], outs_b[l]), l
         for c in range(2):
             assert torch.equal(states_a[c][l], states_b[c][l]), (l, c)
+    del a, outs_a, states_a
     for l in range(R):
-        Sr, q, k, v, beta, g, _ = oracle_inputs(w, tis[l], S0=S0s[l])
+        Sr, q, k, v, beta, g, bon = oracle_inputs(w, tis[l], S0=S0s[l], bonus=bons[l])
         S = Sr
         o = to_np(outs_b[l])
         for c in range(2):
             sl = slice(c * C, (c + 1) * C)
-            S, o_ref = oracle.eager_run(w.op, S, q[sl], k[sl], v[sl], beta[sl], g[sl], None,
-                                        w.scale)
+            S, o_ref = run_oracle_eager(w, S, q[sl], k[sl], v[sl], beta[sl], g[sl], bon)
             for i, t in enumerate(range(c * C, (c + 1) * C)):
                 assert rel_err(o[t], o_ref[i]) <= tol_out(w), (l, t)
             assert rel_err(to_np(states_b[c][l]), S) <= TOL_STATE, (l, c)
