@@ -156,7 +156,8 @@ def test_cycle_staggered_with_empty_layer(op, mode, layout):
 
 
 @pytest.mark.parametrize("name", ["gdn-b128-h16-d128-c8", "kda-b128-h32-d128-c8",
-                                  "rwkv6-b128-h32-d64-c8"])
+                                  "kda-b128-h32-d128-c4", "rwkv6-b128-h32-d64-c8",
+                                  "rwkv6-b128-h32-d64-c4"])
 @pytest.mark.parametrize("mode", MODES)
 def test_cycle_full_size(mode, name):
     """The bench's workloads as four-layer cycles (the bench's step), two
