@@ -108,15 +108,6 @@ struct EagerParams {
 
 // -------------------------------------------------------------- helpers --
 
-__device__ __forceinline__ float4 ld_stream(const float *p) {
-    // read-once state stream: bypass L1, keep the default L2 policy
-    float4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 __device__ __forceinline__ float4 ld_state(const float *p) {
     // state tile that this kernel also writes back (coherent path)
     return *reinterpret_cast<const float4 *>(p);
@@ -138,26 +129,10 @@ __device__ __forceinline__ void st_out(void *p, size_t i, float x, int bf16) {
         reinterpret_cast<float *>(p)[i] = x;
 }
 
-// raw copy of one element of an input vector (bit-exact, either dtype)
-__device__ __forceinline__ void copy_in(void *dst, size_t di, const void *src, size_t si,
-                                        int bf16) {
-    if (bf16)
-        reinterpret_cast<uint16_t *>(dst)[di] = reinterpret_cast<const uint16_t *>(src)[si];
-    else
-        reinterpret_cast<float *>(dst)[di] = reinterpret_cast<const float *>(src)[si];
-}
-
 // element i of a raw vector in shared (or global) memory, either dtype
 __device__ __forceinline__ float ld_raw(const void *p, int i, int bf16) {
     if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
     return reinterpret_cast<const float *>(p)[i];
-}
-
-__device__ __forceinline__ void copy_raw(void *dst, size_t di, const void *src, int si, int bf16) {
-    if (bf16)
-        reinterpret_cast<uint16_t *>(dst)[di] = reinterpret_cast<const uint16_t *>(src)[si];
-    else
-        reinterpret_cast<float *>(dst)[di] = reinterpret_cast<const float *>(src)[si];
 }
 
 // Asynchronous global -> shared copies (sm_80+ cp.async; completion is
@@ -199,21 +174,6 @@ __device__ __forceinline__ float4 ld_stream_hint(const float *p, uint64_t pol) {
                  : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
                  : "l"(p), "l"(pol));
     return r;
-}
-
-__device__ __forceinline__ float4 ld_state_hint(const float *p, uint64_t pol) {
-    float4 r;
-    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
-                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-                 : "l"(p), "l"(pol)
-                 : "memory");
-    return r;
-}
-
-__device__ __forceinline__ void st_state_hint(float *p, float4 v, uint64_t pol) {
-    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
-                 "f"(v.z), "f"(v.w), "l"(pol)
-                 : "memory");
 }
 
 __device__ __forceinline__ void st_f32_hint(float *p, float v, uint64_t pol) {
