@@ -149,3 +149,29 @@ def test_clock_sampler_with_fake_nvml(monkeypatch):
     assert s["samples"] >= 10
     assert s["sm_mhz"] == 1965                  # idle sample left out
     assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    """`--impl reference` (the oracle on the host cores) prints one JSON line
+    with the native arm's config object and the contract's keys; under a
+    launcher, ranks other than 0 print nothing and return."""
+    import json
+    w = "gdn-b1-h2-d64-c4-fp32"
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--workload", w, "--steps", "1", "--warmup", "3"])
+    assert capsys.readouterr().out == ""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.main(["--impl", "reference", "--workload", w, "--steps", "1", "--warmup", "3"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    assert r["impl"] == "reference" and r["value"] > 0 and r["unit"] == "tok/s"
+    assert r["config"] == bench.workload_config(synth.WORKLOADS[w], 4, 1)
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
+    assert r["e2e"] == {"value": r["value"], "unit": "tok/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    for k in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data"):
+        assert k in r
