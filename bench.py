@@ -304,6 +304,31 @@ def working_set(w, R):
     return R * w.heads * (bm["S"] + w.C * bm["E"])
 
 
+def cold_layers(w, R, most=16):
+    """Rotated layers for a workload's cold figures: at least R, and enough
+    that the working set is at least 4x the L2 (at most `most`)."""
+    r = R
+    while working_set(w, r) < 4 * L2_BYTES and r < most:
+        r += 1
+    return r
+
+
+def hot_cycle_us(w, args, dev, stream):
+    """µs per layer-token of one layer's merge cycle decoded over and over,
+    its whole working set resident in L2 (the hot figure beside the cold
+    one; only for workloads whose layer fits in L2)."""
+    from recurrent_state_head_b200 import binding as B
+    rank = int(os.environ.get("RANK", "0"))
+    su = Setup(w, 1, rank, dev)
+    layers = su.layers(B.DL_MERGE_FOLD)
+    outs = [L_.new_out(w.C) for L_ in layers]
+    cyc = B.Cycle([L_.handle for L_ in layers], _ios(w, su.xs, outs, 1, w.C))
+    ms = _time_graph(lambda: cyc.launch(stream), stream, args.steps, args.warmup, dev)
+    ms, _ = reduce_over_ranks(ms / args.steps, 0, dev)
+    cyc.close()
+    return ms * 1e3 / w.C
+
+
 def workload_config(w, R, world):
     """The `config` object of a bench line (the same keys in both arms)."""
     ws = working_set(w, R)
@@ -783,7 +808,8 @@ def run_native(args, rank, world, local_rank):
             if name == w.name:
                 continue
             wx = synth.WORKLOADS[name]
-            r, k = measure(wx, R, args, dev, stream, peaks, headline=False)
+            Rw = cold_layers(wx, R)
+            r, k = measure(wx, Rw, args, dev, stream, peaks, headline=False)
             k["cycle"].close()
             del k
             torch.cuda.empty_cache()
@@ -796,8 +822,11 @@ def run_native(args, rank, world, local_rank):
                 "merge_token_frac": r["kernels"].get("merge_token_frac"),
                 "merge_us": r["kernels"]["merge_us"],
                 "bytes_written_per_token": r["bytes_written_per_token"],
-                "clocks": r["clocks"],
+                "clocks": r["clocks"], "config": workload_config(wx, Rw, world),
             }
+            if working_set(wx, 1) < L2_BYTES:
+                extra[name]["hot_us_per_token"] = hot_cycle_us(wx, args, dev, stream)
+                torch.cuda.empty_cache()
             if "eager" in r:
                 extra[name].update({"eager_us_per_token": r["eager"]["us_per_token"],
                                     "eager_hbm_frac": r["eager"]["hbm_frac"],

@@ -175,3 +175,17 @@ def test_reference_arm_line(monkeypatch, capsys):
     for k in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data"):
         assert k in r
+
+
+def test_cold_rotation_reaches_four_times_l2():
+    """Every workload's cold figures rotate enough layers that the working
+    set is at least 4x the L2; a layer that fits in L2 also gets a hot
+    figure."""
+    for name in (bench.DEFAULT_WORKLOAD,) + bench.EXTRA_WORKLOADS:
+        w = synth.WORKLOADS[name]
+        R = bench.cold_layers(w, 4)
+        assert R >= 4
+        assert bench.working_set(w, R) >= 4 * bench.L2_BYTES
+        assert R == 4 or bench.working_set(w, R - 1) < 4 * bench.L2_BYTES
+    assert bench.cold_layers(synth.WORKLOADS["rwkv6-b128-h32-d64-c8"], 4) == 7
+    assert bench.working_set(synth.WORKLOADS["rwkv6-b128-h32-d64-c8"], 1) < bench.L2_BYTES
